@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV attention step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the host work
+partition (pa_plan_build), the cache write (pa_reshape_and_cache) and varlen
+paged attention (pa_attention_varlen: split-KV decode kernel + combine, and the
+tensor-core prefill kernel when the batch holds long segments).  Inputs are
+seeded and synthetic with the shapes of the named workload (model names give
+attention shapes only; no weights).  Default workload: 64 decodes with the
+TinyLlama-1.1B attention shape.
+
+Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier and
+torch.cuda.synchronize() on both sides.  L2 is flushed (a 512 MiB write)
+before every step and each step's device time is taken with CUDA events on
+the launching stream, excluding the flush; the host plan for a step is built
+while the flush runs.  Multi-GPU (torchrun): every rank runs its own batch of
+the same shape (weak scaling, no collective on the data path); the reported
+time is the max over ranks.
+
+The JSON line adds: roofline (dominant kernel, timed live with CUDA events
+around it), e2e (same metric through the public API with host buffers: H2D of
+the step's inputs and D2H of its output inside the timed region), the CPU
+oracle as a reported baseline, SM clocks sampled during the timed region, and
+the number of library kernels launched.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged-attn decode KV GB/s (% of HBM peak); mixed-batch attn tokens/s, % roofline"
+DEFAULT_WORKLOAD = "decode_tinyllama_b64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 512 << 20
+
+
+# ---------------------------------------------------------------------------
+# accounting
+# ---------------------------------------------------------------------------
+
+def step_bytes(lay: W.Layout) -> dict:
+    """Algorithmic bytes of one step: every distinct KV byte the attention must
+    read once, q read, out written, the scatter's read of k/v and write of the
+    cache rows, and the block-table entries and lengths read."""
+    T, Hq, Hkv, D = lay.num_tokens, lay.num_q_heads, lay.num_kv_heads, lay.head_dim
+    kv = lay.kv_bytes_read()
+    qo = 2 * T * Hq * D * 2
+    scatter = 2 * (2 * T * Hkv * D * 2)
+    used_blocks = int(sum(-(-int(n) // 16) for n in lay.seq_lens))
+    meta = used_blocks * 4 + lay.num_seqs * 8 + T * 8
+    return {"kv": kv, "qo": qo, "scatter": scatter, "meta": meta, "total": kv + qo + scatter + meta}
+
+
+def is_decode_workload(lay: W.Layout) -> bool:
+    return bool(np.all(lay.q_lens <= 1))
+
+
+def dims_for(pa, lay):
+    return pa.Dims(lay.num_tokens, lay.num_seqs, lay.num_q_heads, lay.num_kv_heads,
+                   lay.head_dim, lay.num_blocks, lay.max_blocks_per_seq, 16)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(names) -> str:
+    h = hashlib.sha1()
+    for n in names:
+        with open(os.path.join(ROOT, "paged_kv_attention_token_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "counters.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != src_hash:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled every ~2 ms through NVML in a
+    background thread while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
+        self._h = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+
+    def start(self):
+        import threading
+        try:
+            self._h = self._handle()
+            nv = self._nvml
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            nv = self._nvml
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                    self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def stop(self):
+        if self._thread is None:
+            return None
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(names), "source": "nvml"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reported baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_seqs(lay: W.Layout, budget_macs: float, seed: int = 0):
+    """Segments whose oracle cost fits the budget (all of them if it does)."""
+    cost = []
+    for L, n in zip(lay.q_lens.astype(np.int64), lay.seq_lens.astype(np.int64)):
+        keys = int(L * (n - L) + L * (L + 1) // 2)
+        cost.append(2 * keys * lay.num_q_heads * lay.head_dim)
+    cost = np.array(cost, dtype=np.float64)
+    if cost.sum() <= budget_macs:
+        return list(range(lay.num_seqs)), cost.sum()
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(lay.num_seqs)
+    pick, acc = [], 0.0
+    for i in order:
+        if acc + cost[i] > budget_macs and pick:
+            continue
+        pick.append(int(i))
+        acc += cost[i]
+    return sorted(pick), acc
+
+
+def time_oracle(batch: W.Batch, seconds: float, budget_macs: float):
+    """Run the oracle (scatter + attention) on a bounded sample of the batch
+    until `seconds` have passed; returns per-run seconds and what was run."""
+    import oracle as O
+    lay = batch.layout
+    seqs, _ = oracle_sample_seqs(lay, budget_macs)
+    hs = W.host_subset(batch, seqs)
+    sub = W.Layout(lay.name, lay.num_q_heads, lay.num_kv_heads, lay.head_dim, lay.num_blocks,
+                   lay.q_lens[seqs], lay.seq_lens[seqs], lay.block_tables[seqs], lay.poison_block,
+                   lay.shared_prefix_blocks)
+    threads = O.default_threads()
+    runs = []
+    t_end = time.perf_counter() + seconds
+    while True:
+        kc, vc = hs.k_cache.copy(), hs.v_cache.copy()
+        t0 = time.perf_counter()
+        O.reshape_and_cache(hs.k, hs.v, hs.slot_mapping, kc, vc)
+        O.attention_varlen(hs.q, kc, vc, hs.block_tables, hs.cu_seqlens_q, hs.seq_lens,
+                           batch.scale, threads=threads)
+        runs.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end:
+            break
+    units = {"bytes": step_bytes(sub)["total"] if len(seqs) else 0, "tokens": int(lay.q_lens[seqs].sum()),
+             "seqs": len(seqs)}
+    return runs, units, threads
+
+
+def baseline_value(decode: bool, units: dict, sec: float) -> float:
+    return units["bytes"] / sec / 1e9 if decode else units["tokens"] / sec
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the CPU oracle, as it stands
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    lay = W.layout(args.workload)
+    decode = is_decode_workload(lay)
+    # inputs are drawn on the GPU when there is one (faster for big pools);
+    # only the oracle's host run is timed
+    batch = W.make_batch(lay, device="cuda" if torch.cuda.is_available() else "cpu")
+    per_step = []
+    budget = 2.0e9
+    runs_all = []
+    units = None
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        runs, units, threads = time_oracle(batch, 0.0, budget)
+        if i >= args.warmup:
+            runs_all.extend(runs)
+    sec = statistics.mean(runs_all)
+    value = baseline_value(decode, units, sec)
+    unit = "GB/s" if decode else "tokens/s"
+    sample = (f"{units['seqs']} of {lay.num_seqs} segments ({units['tokens']} query tokens), "
+              "oracle scatter + attention per step")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": args.workload, "shape": lay.description},
+           "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import paged_kv_attention_token_b200 as pa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    pa.load_library()
+
+    fn, default_seed, _ = W.WORKLOADS[args.workload]
+    lay = W.layout(args.workload, seed=default_seed + 7919 * rank)
+    decode = is_decode_workload(lay)
+    batch = W.make_batch(lay, device=dev)
+    acct = step_bytes(lay)
+    bt, cu, sl, slots = batch.device_ints(dev)
+    h_cu, h_sl = lay.cu_seqlens_q, lay.seq_lens
+    kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
+    out = torch.empty_like(batch.q)
+    dims = dims_for(pa, lay)
+    plan0 = pa.Plan(h_cu, h_sl, dims, device=local)
+    info = plan0.info()
+    ws = pa.workspace_for(plan0, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + \
+        (1 if info["num_combine_rows"] else 0) + (1 if info["num_prefill_tiles"] else 0)
+
+    def one_step(trace=None, ev=None):
+        flush.fill_(1)
+        t0 = time.perf_counter()
+        plan = pa.Plan(h_cu, h_sl, dims, device=local)
+        plan_s = time.perf_counter() - t0
+        if ev is not None:
+            ev[0].record(stream)
+        pa.reshape_and_cache(batch.k, batch.v, slots, kc, vc, stream=stream)
+        pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws,
+                            stream=stream, trace=trace)
+        if ev is not None:
+            ev[1].record(stream)
+        return plan, plan_s
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(dev)
+
+    traces = [pa.Trace() for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    plans, plan_times = [], []
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        plan, plan_s = one_step(traces[i], evs[i])
+        plans.append(plan)
+        plan_times.append(plan_s)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    stages = [t.elapsed_ms() for t in traces]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ms_per_step = max_total_ms / args.steps
+
+    if decode:
+        unit = "GB/s"
+        value = world * acct["total"] * args.steps / (max_total_ms * 1e-3) / 1e9
+    else:
+        unit = "tokens/s"
+        value = world * lay.num_tokens * args.steps / (max_total_ms * 1e-3)
+
+    # roofline of the dominant kernel: the split-KV decode kernel
+    peaks, peak_kind = load_peaks()
+    dec_ms = statistics.mean(s["decode"] for s in stages)
+    comb_ms = statistics.mean(s["combine"] for s in stages)
+    copy_ms = statistics.mean(s["table_copy"] for s in stages)
+    dec_bytes = acct["kv"] + acct["qo"] + acct["meta"]
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    src_hash = kernel_source_hash(["decode.cu", "common.cuh", "kernels.h", "plan.h"])
+    roofline = {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": profiled_traffic("decode_kernel", args.workload, src_hash),
+                "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash}
+
+    # e2e: public API with host buffers; H2D of the step's inputs, D2H of out
+    e2e = None
+    if not args.no_e2e:
+        host = {n: x.detach().cpu().pin_memory() for n, x in
+                (("q", batch.q), ("k", batch.k), ("v", batch.v), ("slots", slots),
+                 ("bt", bt), ("cu", cu), ("sl", sl))}
+        dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(x.numel() * x.element_size() for x in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        e_ms = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(2)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for n in host:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            plan = pa.Plan(h_cu, h_sl, dims, device=local)
+            pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)
+            pa.attention_varlen(dev_in["q"], kc, vc, dev_in["bt"], dev_in["cu"], dev_in["sl"],
+                                batch.scale, out, plan, ws, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                e_ms.append(e0.elapsed_time(e1))
+        te = torch.tensor([sum(e_ms)], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e_total = float(te.item())
+        e_val = (world * acct["total"] * args.steps / (e_total * 1e-3) / 1e9) if decode else \
+            (world * lay.num_tokens * args.steps / (e_total * 1e-3))
+        e2e = {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_total / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host_batch = batch
+        runs, units, threads = time_oracle(host_batch, args.cpu_seconds, 2.0e9)
+        sec = statistics.mean(runs)
+        cpu = {"value": baseline_value(decode, units, sec), "unit": unit, "cores": threads,
+               "kind": "oracle",
+               "sample": f"{units['seqs']} of {lay.num_seqs} segments ({units['tokens']} query tokens), "
+                         f"oracle scatter + attention, {len(runs)} runs, mean {sec:.3f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "shape": lay.description,
+                       "bytes_per_step": acct["total"], "kv_bytes_per_step": acct["kv"],
+                       "tokens_per_step": lay.num_tokens,
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)",
+                       "plan_us_host": 1e6 * statistics.median(plan_times),
+                       "stages_ms": {"table_copy": copy_ms, "decode": dec_ms, "combine": comb_ms,
+                                     "prefill": statistics.mean(s["prefill"] for s in stages)},
+                       "parallelism": f"replicas x{world} (weak: one batch per GPU)",
+                       "wall_s_timed_region": wall},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

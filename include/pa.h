@@ -1,0 +1,227 @@
+/*
+ * pa.h — C ABI of libpa.so: the paged-KV attention step of one
+ * continuous-batching forward pass, for NVIDIA B200 (sm_100a).
+ *
+ * The operation follows "vLLM 学习笔记 01：一个请求在 vLLM 里的一生":
+ *   §1.5  the KV cache is cut into fixed 16-token blocks; each request owns a
+ *         block table naming the physical block of each of its logical
+ *         blocks, and the blocks need not be contiguous;
+ *   §1.6  all tokens scheduled in a step are concatenated into one unpadded
+ *         stream; the attention op is told where each segment starts and
+ *         ends (segments cannot see one another), which slot (block and row)
+ *         each new token's K/V is written to, and which blocks hold each
+ *         segment's history; prefill chunks and single-token decodes share
+ *         one batch;
+ *   §1.4  a request tracks computed vs total tokens, so seq_len below counts
+ *         the tokens scheduled in this step, and §2.1: a prefill chunk reads
+ *         the context earlier chunks cached.
+ * The block layout follows "Inside vLLM: Anatomy of a High-Throughput LLM
+ * Inference System" (Chinese translation), section "LLM 引擎构造函数": a block
+ * of a standard layer holds K and V of block_size tokens for every kv head.
+ *
+ * Conventions for every call
+ *  - Pointers named d_* or described as "device" are CUDA device pointers on
+ *    the current device; h_* pointers are host memory.  The caller owns every
+ *    buffer and keeps it alive until the work queued on `stream` completes.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    are asynchronous on it unless stated otherwise.
+ *  - bf16 tensors are row-major and contiguous, base addresses 16-byte
+ *    aligned.  Shapes (T = num_tokens, S = num_seqs, Hq, Hkv, D = head_dim,
+ *    NB = num_blocks, MB = max_blocks_per_seq, B = block_size):
+ *        q, out        [T][Hq][D]      bf16
+ *        k, v          [T][Hkv][D]     bf16
+ *        k_cache       [NB][B][Hkv][D] bf16   (v_cache the same, separate)
+ *        block_tables  [S][MB]         int32
+ *        cu_seqlens_q  [S+1]           int32  (0, non-decreasing, ends at T)
+ *        seq_lens      [S]             int32  (q_len <= seq_len)
+ *        slot_mapping  [T]             int64
+ *  - Supported: B == 16, D in {64, 128}, Hq % Hkv == 0, Hq / Hkv <= 16.
+ *  - Every call returns a pa_status and never aborts, throws or traps.
+ *    Violations checkable on the host (null pointers, sizes, alignment,
+ *    unsupported shapes, workspace too small) are rejected before any work
+ *    is queued.  Data-dependent preconditions (slots and block ids inside
+ *    the pool, q_len <= seq_len, distinct slots, the device arrays agreeing
+ *    with the host arrays the plan was built from) are not checked by the
+ *    compute calls; pa_validate_inputs checks them on request.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_NULL = -1,        /* a required pointer is NULL */
+    PA_ERR_SHAPE = -2,       /* inconsistent or negative sizes */
+    PA_ERR_DTYPE = -3,       /* reserved: the binding reports wrong dtypes with it */
+    PA_ERR_ALIGN = -4,       /* a base address is not 16-byte aligned */
+    PA_ERR_UNSUPPORTED = -5, /* block_size != 16, head_dim not 64/128, group > 16 */
+    PA_ERR_WORKSPACE = -6,   /* workspace NULL or smaller than the plan needs */
+    PA_ERR_BOUNDS = -7,      /* pa_validate_inputs found a precondition violated */
+    PA_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
+    PA_ERR_PLAN = -9         /* the plan does not match the dims of the call */
+} pa_status;
+
+/* Sizes of one call.  block_size must be 16. */
+typedef struct {
+    int32_t num_tokens;          /* T: scheduled tokens in the flat stream */
+    int32_t num_seqs;            /* S: segments (requests) */
+    int32_t num_q_heads;         /* Hq */
+    int32_t num_kv_heads;        /* Hkv; query head h reads kv head h / (Hq/Hkv) */
+    int32_t head_dim;            /* D: 64 or 128 */
+    int32_t num_blocks;          /* NB: blocks in the pool */
+    int32_t max_blocks_per_seq;  /* MB: columns of block_tables */
+    int32_t block_size;          /* B: tokens per block, must be 16 */
+} pa_dims;
+
+/*
+ * reshape_and_cache — "vLLM 学习笔记 01" §1.6: each new token's K/V is
+ * written to the slot its slot mapping names.  For every t in [0, T) with
+ * s = slot_mapping[t] >= 0: k_cache[s / 16][s % 16][:][:] = k[t][:][:] and
+ * v_cache likewise, bit for bit.  A negative slot skips the token.  Nothing
+ * else in the caches changes.
+ *   d_k, d_v              device [T][Hkv][D] bf16, read
+ *   d_slot_mapping        device [T] int64, read; each s < NB * 16 and no two
+ *                         tokens share a slot (precondition)
+ *   d_k_cache, d_v_cache  device [NB][16][Hkv][D] bf16, written in place
+ *   dims                  host; num_seqs, num_q_heads, max_blocks_per_seq unused
+ * T == 0 queues nothing and returns PA_OK.
+ */
+int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot_mapping,
+                         void *d_k_cache, void *d_v_cache, const pa_dims *dims,
+                         void *stream);
+
+/*
+ * Work partition for pa_attention_varlen (host only; queues no GPU work).
+ * From the host copies of cu_seqlens_q and seq_lens (the same values the
+ * device arrays will hold) it splits the step into balanced GPU work:
+ * segments with q_len <= 16 (decodes, speculative-verification shapes) are
+ * cut into equal runs of 16-token KV blocks over all query rows and kv heads
+ * (split-KV), each run one warp's work, with a combine step for rows cut in
+ * several runs; longer segments are cut into 128-query tiles per query head
+ * for the tensor-core prefill kernel, longest tiles first.
+ *   h_cu_seqlens_q  host [S+1] int32
+ *   h_seq_lens      host [S] int32
+ *   dims            host; T, S, Hq, Hkv, D, B are used
+ *   device          CUDA device ordinal the plan is sized for (its SM count
+ *                   is read once per process and cached; -1 = assume 148 SMs)
+ *   out             receives a new plan owned by the caller; free it with
+ *                   pa_plan_destroy.  A plan is immutable and may be reused
+ *                   for every layer of a step, and by several streams.
+ * Errors: PA_ERR_NULL, PA_ERR_SHAPE (cu_seqlens not starting at 0, not
+ * non-decreasing or not ending at T; q_len > seq_len), PA_ERR_UNSUPPORTED.
+ */
+typedef struct pa_plan pa_plan;
+int pa_plan_build(const int32_t *h_cu_seqlens_q, const int32_t *h_seq_lens,
+                  const pa_dims *dims, int device, pa_plan **out);
+
+/* What a plan holds, for tests, logging and roofline accounting. */
+typedef struct {
+    int32_t num_sms;              /* SM count the plan was sized for */
+    int32_t num_decode_rows;      /* (query token, kv head) rows on the split-KV path */
+    int32_t num_decode_units;     /* warps of the split-KV kernel */
+    int32_t num_partials;         /* partial results the combine step merges */
+    int32_t num_combine_rows;     /* rows cut across more than one warp */
+    int32_t num_prefill_tiles;    /* (128-query tile, query head) items */
+    int64_t decode_kv_blocks;     /* sum over decode rows of ceil(keys / 16) */
+    int64_t prefill_causal_pairs; /* (query, visible key) pairs per query head */
+    uint64_t table_bytes;         /* plan tables copied into the workspace per call */
+    uint64_t workspace_bytes;     /* = pa_plan_workspace_bytes */
+} pa_plan_info;
+int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
+
+/* Bytes of device workspace pa_attention_varlen needs with this plan
+ * (0 for a NULL plan).  256-byte alignment of the workspace is required. */
+size_t pa_plan_workspace_bytes(const pa_plan *plan);
+
+/* Frees a plan (NULL is allowed).  Work already queued that used the plan is
+ * not affected: the plan's tables are copied into the workspace when the
+ * call is queued. */
+void pa_plan_destroy(pa_plan *plan);
+
+/*
+ * Varlen paged attention — "vLLM 学习笔记 01" §1.5-§1.6, §2.1.  For every
+ * segment i with q_len L = cu_seqlens_q[i+1] - cu_seqlens_q[i] and seq_len n,
+ * query j (0 <= j < L, flat token t = cu_seqlens_q[i] + j) sits at position
+ * p = n - L + j (bottom-right causal alignment) and, for every query head h
+ * with kv head g = h / (Hq / Hkv):
+ *     z_tau  = scale * <q[t][h], K_i[tau][g]>            tau = 0 .. p
+ *     out[t][h] = sum_tau softmax(z)_tau * V_i[tau][g]
+ * where K_i[tau] = k_cache[block_tables[i][tau / 16]][tau % 16] (V alike).
+ * Block-table entries past ceil(n / 16) and cache rows past n are never read.
+ * Arithmetic: bf16 operands, fp32 accumulation and online softmax, output
+ * rounded to bf16 (round to nearest even).  The new tokens are read from the
+ * cache, so pa_reshape_and_cache for this step must be queued first.
+ *   d_q             device [T][Hq][D] bf16
+ *   d_k_cache/d_v_cache  device [NB][16][Hkv][D] bf16
+ *   d_block_tables  device [S][MB] int32
+ *   d_cu_seqlens_q  device [S+1] int32, equal to the host copy given to plan
+ *   d_seq_lens      device [S] int32, equal to the host copy given to plan
+ *   scale           softmax scale (usually 1/sqrt(D))
+ *   d_out           device [T][Hq][D] bf16, written
+ *   plan            from pa_plan_build with the same dims
+ *   d_workspace     device scratch of pa_plan_workspace_bytes(plan) bytes,
+ *                   256-byte aligned; the plan tables are copied into it on
+ *                   `stream` and the split partials live there.  Two calls
+ *                   in flight at once need two workspaces.
+ * Errors: PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_UNSUPPORTED,
+ * PA_ERR_PLAN, PA_ERR_WORKSPACE, PA_ERR_CUDA.
+ */
+int pa_attention_varlen(const void *d_q, const void *d_k_cache, const void *d_v_cache,
+                        const int32_t *d_block_tables, const int32_t *d_cu_seqlens_q,
+                        const int32_t *d_seq_lens, float scale, void *d_out,
+                        const pa_dims *dims, const pa_plan *plan, void *d_workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * pa_attention_varlen with optional tracing: when `trace` is not NULL, each
+ * non-NULL entry of trace->events (a cudaEvent_t created by the caller) is
+ * recorded on `stream` at a fixed point of the call, so that the caller can
+ * time every kernel on the stream it runs on:
+ *   [0] before the plan-table copy     [1] before the split-KV decode kernel
+ *   [2] after the split-KV kernel      [3] after the combine kernel
+ *   [4] before the prefill kernel      [5] after the prefill kernel
+ * Events of stages that do not run are still recorded (adjacent), so every
+ * interval is defined.  Results are identical to pa_attention_varlen.
+ */
+typedef struct {
+    void *events[6];
+} pa_trace;
+int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d_v_cache,
+                           const int32_t *d_block_tables, const int32_t *d_cu_seqlens_q,
+                           const int32_t *d_seq_lens, float scale, void *d_out,
+                           const pa_dims *dims, const pa_plan *plan, void *d_workspace,
+                           size_t workspace_bytes, void *stream, const pa_trace *trace);
+
+/*
+ * Opt-in check of the data-dependent preconditions, on the device, then a
+ * synchronize of `stream`: every slot_mapping entry is negative or inside the
+ * pool; no two tokens share a slot; cu_seqlens_q starts at 0, is
+ * non-decreasing and ends at T; 0 <= q_len <= seq_len; seq_len <= MB * 16;
+ * every block-table entry a segment reads (the first ceil(seq_len / 16)) is
+ * inside the pool.  d_slot_mapping may be NULL to skip the slot checks.
+ * Returns PA_OK, PA_ERR_BOUNDS, or a host-side error as above.
+ *   d_scratch  device, at least pa_validate_scratch_bytes(dims) bytes,
+ *              256-byte aligned (overwritten).
+ */
+size_t pa_validate_scratch_bytes(const pa_dims *dims);
+int pa_validate_inputs(const int64_t *d_slot_mapping, const int32_t *d_block_tables,
+                       const int32_t *d_cu_seqlens_q, const int32_t *d_seq_lens,
+                       const pa_dims *dims, void *d_scratch, size_t scratch_bytes,
+                       void *stream);
+
+/* Static text for a status code. */
+const char *pa_status_string(int status);
+
+/* Library version, e.g. "0.1.0". */
+const char *pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA_H */

@@ -1,0 +1,292 @@
+"""Python binding of libpa.so, the paged-KV attention step for B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/pa.h.  There is no CPU or
+PyTorch fallback; if the library is missing or cannot be loaded, every call
+raises.  PyTorch supplies device memory and streams.
+
+    import paged_kv_attention_token_b200 as pa
+    pa.reshape_and_cache(k, v, slot_mapping, k_cache, v_cache)
+    plan = pa.Plan(cu_seqlens_q_host, seq_lens_host, pa.dims_of(q, k_cache, block_tables, seq_lens))
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    pa.attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens,
+                        scale, out, plan, ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+__all__ = ["load_library", "library_path", "PaError", "Dims", "dims_of", "Plan",
+           "reshape_and_cache", "attention_varlen", "validate_inputs", "status_string", "Trace",
+           "workspace_for",
+           "PA_OK", "PA_ERR_NULL", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "PA_ERR_ALIGN",
+           "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_BOUNDS", "PA_ERR_CUDA", "PA_ERR_PLAN"]
+
+PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE, PA_ERR_ALIGN = 0, -1, -2, -3, -4
+PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_BOUNDS, PA_ERR_CUDA, PA_ERR_PLAN = -5, -6, -7, -8, -9
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libpa.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = status_string(status) if _lib is not None else str(status)
+        super().__init__(f"{what}: {msg} (status {status})" if what else f"{msg} (status {status})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_tokens", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("block_size", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "Dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_sms", ctypes.c_int32), ("num_decode_rows", ctypes.c_int32),
+                ("num_decode_units", ctypes.c_int32), ("num_partials", ctypes.c_int32),
+                ("num_combine_rows", ctypes.c_int32), ("num_prefill_tiles", ctypes.c_int32),
+                ("decode_kv_blocks", ctypes.c_int64), ("prefill_causal_pairs", ctypes.c_int64),
+                ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64)]
+
+    def as_dict(self):
+        return {n: int(getattr(self, n)) for n, _ in self._fields_}
+
+
+def load_library():
+    """Load libpa.so (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library {_LIB_PATH} is missing: build it with "
+                               "`python -m paged_kv_attention_token_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, SZ, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        DP = ctypes.POINTER(Dims)
+        sig = {
+            "pa_reshape_and_cache": (I, [P, P, P, P, P, DP, P]),
+            "pa_plan_build": (I, [P, P, DP, I, ctypes.POINTER(P)]),
+            "pa_plan_get_info": (I, [P, ctypes.POINTER(PlanInfo)]),
+            "pa_plan_workspace_bytes": (SZ, [P]),
+            "pa_plan_destroy": (None, [P]),
+            "pa_attention_varlen": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P]),
+            "pa_attention_varlen_ex": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P, P]),
+            "pa_validate_scratch_bytes": (SZ, [DP]),
+            "pa_validate_inputs": (I, [P, P, P, P, DP, P, SZ, P]),
+            "pa_status_string": (ctypes.c_char_p, [I]),
+            "pa_version": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().pa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PaError(status, what)
+
+
+def _dev_ptr(t: torch.Tensor | None, name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise PaError(PA_ERR_SHAPE, f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise PaError(PA_ERR_DTYPE, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise PaError(PA_ERR_SHAPE, f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def dims_of(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor,
+            seq_lens) -> Dims:
+    """Dims of a call from the tensors' shapes (q [T,Hq,D], cache [NB,16,Hkv,D],
+    block_tables [S,MB])."""
+    T, Hq, D = q.shape
+    NB, B, Hkv, D2 = k_cache.shape
+    if D2 != D:
+        raise PaError(PA_ERR_SHAPE, "q and cache head_dim differ")
+    S = len(seq_lens)
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    return Dims(T, S, Hq, Hkv, D, NB, MB, B)
+
+
+def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                      k_cache: torch.Tensor, v_cache: torch.Tensor, stream=None) -> None:
+    """Write k[t], v[t] into the caches at slot_mapping[t] (pa_reshape_and_cache)."""
+    lib = load_library()
+    T, Hkv, D = k.shape
+    if v.shape != k.shape or k_cache.shape != v_cache.shape or tuple(k_cache.shape[2:]) != (Hkv, D):
+        raise PaError(PA_ERR_SHAPE, "reshape_and_cache shapes")
+    if slot_mapping.shape != (T,):
+        raise PaError(PA_ERR_SHAPE, "slot_mapping must be [T]")
+    d = Dims(T, 0, Hkv, Hkv, D, k_cache.shape[0], 0, k_cache.shape[1])
+    bf = torch.bfloat16
+    _check(lib.pa_reshape_and_cache(_dev_ptr(k, "k", bf), _dev_ptr(v, "v", bf),
+                                    _dev_ptr(slot_mapping, "slot_mapping", torch.int64),
+                                    _dev_ptr(k_cache, "k_cache", bf), _dev_ptr(v_cache, "v_cache", bf),
+                                    ctypes.byref(d), _stream_ptr(stream)), "pa_reshape_and_cache")
+
+
+def _host_i32(a, name):
+    if isinstance(a, torch.Tensor):
+        if a.is_cuda:
+            raise PaError(PA_ERR_SHAPE, f"{name} must be a host array for planning")
+        a = a.numpy()
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+class Plan:
+    """Work partition for one step (pa_plan_build); reusable for every layer."""
+
+    def __init__(self, cu_seqlens_q, seq_lens, dims: Dims, device: int | None = None):
+        lib = load_library()
+        self._lib = lib
+        self._cu = _host_i32(cu_seqlens_q, "cu_seqlens_q")
+        self._sl = _host_i32(seq_lens, "seq_lens")
+        self.dims = Dims(*[getattr(dims, n) for n, _ in Dims._fields_])
+        if device is None:
+            device = torch.cuda.current_device() if torch.cuda.is_available() else -1
+        h = ctypes.c_void_p()
+        _check(lib.pa_plan_build(self._cu.ctypes.data_as(ctypes.c_void_p),
+                                 self._sl.ctypes.data_as(ctypes.c_void_p), ctypes.byref(self.dims),
+                                 int(device), ctypes.byref(h)), "pa_plan_build")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self._lib.pa_plan_workspace_bytes(self._h))
+
+    def info(self) -> dict:
+        inf = PlanInfo()
+        _check(self._lib.pa_plan_get_info(self._h, ctypes.byref(inf)), "pa_plan_get_info")
+        return inf.as_dict()
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.pa_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def workspace_for(plan: Plan, device=None) -> torch.Tensor:
+    """A device workspace of the size a plan needs (256-byte aligned by torch)."""
+    return torch.empty(max(plan.workspace_bytes, 1), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+class Trace(ctypes.Structure):
+    """Events recorded around the kernels of one attention call (pa_trace)."""
+    _fields_ = [("events", ctypes.c_void_p * 6)]
+
+    STAGES = ("table_copy", "decode", "combine", "gap", "prefill")
+
+    def __init__(self):
+        super().__init__()
+        self.torch_events = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for i, e in enumerate(self.torch_events):
+            self.events[i] = ctypes.c_void_p(e.cuda_event)
+
+    def arm(self, stream):
+        # torch only reports elapsed times of events it has recorded itself;
+        # record them once here, the library records them again at its marks
+        # (the latest record on the stream sets an event's timestamp).
+        for e in self.torch_events:
+            e.record(stream)
+
+    def elapsed_ms(self) -> dict:
+        """Per-stage times (ms) once the stream has reached the last event."""
+        ev = self.torch_events
+        return {"table_copy": ev[0].elapsed_time(ev[1]), "decode": ev[1].elapsed_time(ev[2]),
+                "combine": ev[2].elapsed_time(ev[3]), "prefill": ev[4].elapsed_time(ev[5]),
+                "total": ev[0].elapsed_time(ev[5])}
+
+
+def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale,
+                     out, plan: Plan, workspace: torch.Tensor, stream=None,
+                     trace: "Trace | None" = None) -> torch.Tensor:
+    """Varlen causal paged attention (pa_attention_varlen); writes and returns out.
+    With ``trace``, CUDA events are recorded around each kernel."""
+    lib = load_library()
+    d = plan.dims
+    bf = torch.bfloat16
+    if tuple(q.shape) != (d.num_tokens, d.num_q_heads, d.head_dim) or out.shape != q.shape:
+        raise PaError(PA_ERR_SHAPE, "q/out shape does not match the plan")
+    if tuple(k_cache.shape) != (d.num_blocks, d.block_size, d.num_kv_heads, d.head_dim) or \
+            v_cache.shape != k_cache.shape:
+        raise PaError(PA_ERR_SHAPE, "cache shape does not match the plan")
+    if tuple(block_tables.shape) != (d.num_seqs, d.max_blocks_per_seq):
+        raise PaError(PA_ERR_SHAPE, "block_tables shape does not match the plan")
+    if workspace.dtype != torch.uint8:
+        raise PaError(PA_ERR_DTYPE, "workspace must be uint8")
+    args = (_dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf), _dev_ptr(v_cache, "v_cache", bf),
+            _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(cu_seqlens_q, "cu_seqlens_q", torch.int32),
+            _dev_ptr(seq_lens, "seq_lens", torch.int32),
+            ctypes.c_float(scale), _dev_ptr(out, "out", bf), ctypes.byref(d), plan.handle,
+            _dev_ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel()), _stream_ptr(stream))
+    if trace is None:
+        _check(lib.pa_attention_varlen(*args), "pa_attention_varlen")
+    else:
+        trace.arm(stream if stream is not None else torch.cuda.current_stream())
+        _check(lib.pa_attention_varlen_ex(*args, ctypes.byref(trace)), "pa_attention_varlen_ex")
+    return out
+
+
+def validate_inputs(slot_mapping, block_tables, cu_seqlens_q, seq_lens, dims: Dims,
+                    stream=None) -> int:
+    """Device check of the data-dependent preconditions; returns PA_OK or
+    PA_ERR_BOUNDS (synchronizes the stream)."""
+    lib = load_library()
+    nbytes = int(lib.pa_validate_scratch_bytes(ctypes.byref(dims)))
+    scratch = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=cu_seqlens_q.device)
+    st = lib.pa_validate_inputs(_dev_ptr(slot_mapping, "slot_mapping", torch.int64),
+                                _dev_ptr(block_tables, "block_tables", torch.int32),
+                                _dev_ptr(cu_seqlens_q, "cu_seqlens_q", torch.int32),
+                                _dev_ptr(seq_lens, "seq_lens", torch.int32), ctypes.byref(dims),
+                                _dev_ptr(scratch, "scratch"), ctypes.c_size_t(nbytes),
+                                _stream_ptr(stream))
+    if st not in (PA_OK, PA_ERR_BOUNDS):
+        _check(st, "pa_validate_inputs")
+    return int(st)

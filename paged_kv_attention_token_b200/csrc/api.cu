@@ -1,0 +1,282 @@
+// C ABI of libpa.so: argument checks, plan/workspace plumbing and launches.
+// The declarations, with the meaning of every argument, are in include/pa.h.
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common_dims(const pa_dims *d) {
+    if (!d) return PA_ERR_NULL;
+    if (d->num_tokens < 0 || d->num_seqs < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+        d->head_dim <= 0 || d->num_blocks <= 0 || d->max_blocks_per_seq < 0 || d->block_size <= 0)
+        return PA_ERR_SHAPE;
+    if (d->num_q_heads % d->num_kv_heads != 0) return PA_ERR_SHAPE;
+    if (d->block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (d->num_q_heads / d->num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+int current_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    return device_sm_count(dev);
+}
+
+}  // namespace
+
+int device_sm_count(int device) {
+    if (device < 0 || device >= kMaxDevices) return 148;
+    int v = g_sm_count[device].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // clear the sticky-free error so later calls are not blamed
+        return 148;
+    }
+    g_sm_count[device].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+bool prefill_kernel_available() { return false; }
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" const char *pa_version(void) { return "0.1.0"; }
+
+extern "C" const char *pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "ok";
+        case PA_ERR_NULL: return "a required pointer is NULL";
+        case PA_ERR_SHAPE: return "inconsistent or negative sizes";
+        case PA_ERR_DTYPE: return "wrong dtype";
+        case PA_ERR_ALIGN: return "a base address is not 16-byte aligned";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape (block_size 16, head_dim 64/128, group <= 16)";
+        case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case PA_ERR_BOUNDS: return "input precondition violated (slot, block id or segment bounds)";
+        case PA_ERR_CUDA: return "CUDA error";
+        case PA_ERR_PLAN: return "plan does not match the call";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int pa_reshape_and_cache(const void *k, const void *v, const int64_t *slot_mapping,
+                                    void *k_cache, void *v_cache, const pa_dims *dims,
+                                    void *stream) {
+    if (!dims) return PA_ERR_NULL;
+    const pa_dims &d = *dims;
+    if (d.num_tokens < 0 || d.num_kv_heads <= 0 || d.head_dim <= 0 || d.num_blocks <= 0 ||
+        d.block_size <= 0)
+        return PA_ERR_SHAPE;
+    if (d.block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (d.head_dim != 64 && d.head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (d.num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PA_ERR_ALIGN;
+    const cudaError_t e = launch_reshape_and_cache(
+        k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
+        (int64_t)d.num_blocks * d.block_size, current_sm_count(),
+        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+namespace {
+inline cudaError_t mark(const pa_trace *trace, int i, cudaStream_t stream) {
+    if (!trace || !trace->events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(trace->events[i]), stream);
+}
+}  // namespace
+
+extern "C" int pa_attention_varlen(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_tables, const int32_t *cu_seqlens_q,
+                                   const int32_t *seq_lens, float scale, void *out,
+                                   const pa_dims *dims, const pa_plan *plan, void *workspace,
+                                   size_t workspace_bytes, void *stream_) {
+    return pa_attention_varlen_ex(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale,
+                                  out, dims, plan, workspace, workspace_bytes, stream_, nullptr);
+}
+
+extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const void *v_cache,
+                                      const int32_t *block_tables, const int32_t *cu_seqlens_q,
+                                      const int32_t *seq_lens, float scale, void *out,
+                                      const pa_dims *dims, const pa_plan *plan, void *workspace,
+                                      size_t workspace_bytes, void *stream_, const pa_trace *trace) {
+    int st = check_common_dims(dims);
+    if (st != PA_OK) return st;
+    if (!plan) return PA_ERR_NULL;
+    const pa_dims &d = *dims;
+    const pa_dims &pd = plan->dims;
+    if (pd.num_tokens != d.num_tokens || pd.num_seqs != d.num_seqs ||
+        pd.num_q_heads != d.num_q_heads || pd.num_kv_heads != d.num_kv_heads ||
+        pd.head_dim != d.head_dim || pd.block_size != d.block_size)
+        return PA_ERR_PLAN;
+    if (d.num_tokens == 0) return PA_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !cu_seqlens_q || !seq_lens || !out)
+        return PA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return PA_ERR_ALIGN;
+    const WorkspaceLayout &w = plan->ws;
+    if (w.total > 0) {
+        if (!workspace || workspace_bytes < w.total) return PA_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
+    }
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (w.table_bytes > 0) {
+        // Pageable source: the runtime stages it before returning, so the plan
+        // may be destroyed or rebuilt as soon as this call returns.
+        if (cudaMemcpyAsync(ws, plan->tables.data(), w.table_bytes, cudaMemcpyHostToDevice,
+                            stream) != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
+    const float scale_log2 = scale * kLog2e;
+    if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (plan->num_units > 0) {
+        DecodeParams p;
+        p.q = static_cast<const __nv_bfloat16 *>(q);
+        p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+        p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+        p.block_tables = block_tables;
+        p.out = static_cast<__nv_bfloat16 *>(out);
+        p.partial_o = reinterpret_cast<float *>(ws + w.partial_o);
+        p.partial_ml = reinterpret_cast<float2 *>(ws + w.partial_ml);
+        p.units = reinterpret_cast<const DecodeUnit *>(ws + w.units);
+        p.rows = reinterpret_cast<const DecodeRow *>(ws + w.rows);
+        p.num_units = plan->num_units;
+        p.num_q_heads = d.num_q_heads;
+        p.num_kv_heads = d.num_kv_heads;
+        p.group = plan->group;
+        p.max_blocks_per_seq = d.max_blocks_per_seq;
+        p.scale_log2 = scale_log2;
+        if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 2, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_combine(reinterpret_cast<const CombineRow *>(ws + w.combine), p.rows,
+                           p.partial_o, p.partial_ml, p.out, plan->num_combine, plan->group,
+                           d.num_q_heads, d.num_kv_heads, d.head_dim, stream) != cudaSuccess)
+            return PA_ERR_CUDA;
+    } else if (mark(trace, 2, stream) != cudaSuccess) {
+        return PA_ERR_CUDA;
+    }
+    if (mark(trace, 3, stream) != cudaSuccess || mark(trace, 4, stream) != cudaSuccess ||
+        mark(trace, 5, stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// pa_validate_inputs
+// ---------------------------------------------------------------------------
+
+namespace pa {
+
+__global__ void validate_kernel(const int64_t *__restrict__ slots, const int32_t *__restrict__ bt,
+                                const int32_t *__restrict__ cu, const int32_t *__restrict__ seq,
+                                pa_dims d, uint32_t *__restrict__ bitmap, uint32_t *__restrict__ flag) {
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t num_slots = (int64_t)d.num_blocks * d.block_size;
+    if (slots) {
+        for (int64_t t = tid; t < d.num_tokens; t += stride) {
+            const int64_t s = slots[t];
+            if (s < 0) continue;
+            if (s >= num_slots) {
+                atomicOr(flag, 1u);
+                continue;
+            }
+            const uint32_t bit = 1u << (s & 31);
+            if (atomicOr(bitmap + (s >> 5), bit) & bit) atomicOr(flag, 2u);  // duplicate slot
+        }
+    }
+    for (int64_t i = tid; i < d.num_seqs; i += stride) {
+        const int32_t L = cu[i + 1] - cu[i];
+        if (i == 0 && cu[0] != 0) atomicOr(flag, 4u);
+        if (i == d.num_seqs - 1 && cu[d.num_seqs] != d.num_tokens) atomicOr(flag, 4u);
+        if (L < 0 || seq[i] < L) {
+            atomicOr(flag, 4u);
+            continue;
+        }
+        if (L == 0) continue;
+        const int64_t nb = ((int64_t)seq[i] + d.block_size - 1) / d.block_size;
+        if (nb > d.max_blocks_per_seq) {
+            atomicOr(flag, 8u);
+            continue;
+        }
+        for (int64_t b = 0; b < nb; ++b) {
+            const int32_t id = bt[i * (int64_t)d.max_blocks_per_seq + b];
+            if (id < 0 || id >= d.num_blocks) {
+                atomicOr(flag, 8u);
+                break;
+            }
+        }
+    }
+}
+
+cudaError_t launch_validate(const int64_t *slots, const int32_t *block_tables,
+                            const int32_t *cu_seqlens_q, const int32_t *seq_lens, const pa_dims &d,
+                            uint32_t *slot_bitmap, size_t bitmap_words, uint32_t *flag,
+                            cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return e;
+    if (slots && bitmap_words) {
+        e = cudaMemsetAsync(slot_bitmap, 0, bitmap_words * sizeof(uint32_t), stream);
+        if (e != cudaSuccess) return e;
+    }
+    const int threads = 256;
+    int64_t work = d.num_tokens > d.num_seqs ? d.num_tokens : d.num_seqs;
+    int64_t blocks = (work + threads - 1) / threads;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4096) blocks = 4096;
+    validate_kernel<<<(unsigned)blocks, threads, 0, stream>>>(slots, block_tables, cu_seqlens_q,
+                                                              seq_lens, d, slot_bitmap, flag);
+    return cudaGetLastError();
+}
+
+}  // namespace pa
+
+extern "C" size_t pa_validate_scratch_bytes(const pa_dims *d) {
+    if (!d || d->num_blocks <= 0 || d->block_size <= 0) return 0;
+    const size_t words = ((size_t)d->num_blocks * d->block_size + 31) / 32;
+    return 256 + words * sizeof(uint32_t);
+}
+
+extern "C" int pa_validate_inputs(const int64_t *slot_mapping, const int32_t *block_tables,
+                                  const int32_t *cu_seqlens_q, const int32_t *seq_lens,
+                                  const pa_dims *dims, void *scratch, size_t scratch_bytes,
+                                  void *stream_) {
+    int st = check_common_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims &d = *dims;
+    if (!cu_seqlens_q || !seq_lens || (d.num_seqs > 0 && !block_tables)) return PA_ERR_NULL;
+    if (!scratch || scratch_bytes < pa_validate_scratch_bytes(dims) ||
+        reinterpret_cast<uintptr_t>(scratch) % kWorkspaceAlign)
+        return PA_ERR_WORKSPACE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    uint32_t *flag = static_cast<uint32_t *>(scratch);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(scratch) + 256);
+    const size_t words = ((size_t)d.num_blocks * d.block_size + 31) / 32;
+    if (launch_validate(slot_mapping, block_tables, cu_seqlens_q, seq_lens, d, bitmap, words, flag,
+                        stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+    uint32_t h_flag = 0;
+    if (cudaMemcpyAsync(&h_flag, flag, sizeof h_flag, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+    return h_flag ? PA_ERR_BOUNDS : PA_OK;
+}

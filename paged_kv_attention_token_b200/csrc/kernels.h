@@ -1,0 +1,47 @@
+// Kernel launchers of libpa.so (internal).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "plan.h"
+
+namespace pa {
+
+struct DecodeParams {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_cache;
+    const __nv_bfloat16 *v_cache;
+    const int32_t *block_tables;
+    __nv_bfloat16 *out;
+    float *partial_o;       // [pieces][G][D]
+    float2 *partial_ml;     // [pieces][G]: (max in log2 units, sum)
+    const DecodeUnit *units;
+    const DecodeRow *rows;
+    int num_units;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;
+    int max_blocks_per_seq;
+    float scale_log2;
+};
+
+cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t *slots,
+                                     void *k_cache, void *v_cache, int64_t num_tokens,
+                                     int token_elems, int64_t num_slots, int num_sms,
+                                     cudaStream_t stream);
+
+cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);
+
+cudaError_t launch_combine(const CombineRow *combine, const DecodeRow *rows, const float *partial_o,
+                           const float2 *partial_ml, __nv_bfloat16 *out, int num_combine,
+                           int group, int num_q_heads, int num_kv_heads, int head_dim,
+                           cudaStream_t stream);
+
+// Data-dependent precondition checks; writes a nonzero flag word on failure.
+cudaError_t launch_validate(const int64_t *slots, const int32_t *block_tables,
+                            const int32_t *cu_seqlens_q, const int32_t *seq_lens,
+                            const pa_dims &d, uint32_t *slot_bitmap, size_t bitmap_words,
+                            uint32_t *flag, cudaStream_t stream);
+
+}  // namespace pa

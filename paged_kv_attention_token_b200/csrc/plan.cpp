@@ -1,0 +1,193 @@
+// Host work partitioner: cu_seqlens_q + seq_lens (host copies) -> balanced GPU
+// work.  Pure host code; it queues no GPU work.
+//
+// Decode side (segments with q_len <= kDecodeMaxQLen): every query token of
+// such a segment, for every kv head, is a "row" that reads its p + 1 keys
+// ("vLLM 学习笔记 01" §1.4/§1.6: the segment's seq_len counts this step's
+// tokens, query j sits at position seq_len - q_len + j).  The rows' 16-token
+// KV blocks are laid end to end and cut into equal runs, one run per warp
+// (split-KV in the flash-decoding manner, balanced like stream-K), so every
+// warp moves the same number of KV bytes whatever the length mix.  A row cut
+// across several runs leaves one partial (unnormalised O, running max and
+// sum) per run; the combine step merges them.
+//
+// Prefill side (longer segments): 128-query tiles per query head, ordered by
+// the number of 128-key tiles they read, longest first.
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "plan.h"
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Fewest KV blocks one decode warp is given, so that per-warp fixed costs
+// (loading q, the final write) stay small against the streaming.
+constexpr int64_t kMinBlocksPerUnit = 4;
+
+int check_dims(const pa_dims *d) {
+    if (!d) return PA_ERR_NULL;
+    if (d->num_tokens < 0 || d->num_seqs < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+        d->head_dim <= 0 || d->num_blocks <= 0 || d->max_blocks_per_seq < 0 || d->block_size <= 0)
+        return PA_ERR_SHAPE;
+    if (d->num_q_heads % d->num_kv_heads != 0) return PA_ERR_SHAPE;
+    if (d->block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (d->head_dim != 64 && d->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (d->num_q_heads / d->num_kv_heads > 16) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace
+
+namespace pa {
+int decode_warps_per_sm(int head_dim) { return head_dim <= 64 ? 16 : 8; }
+}  // namespace pa
+
+extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa_dims *dims,
+                             int device, pa_plan **out) {
+    if (!out) return PA_ERR_NULL;
+    *out = nullptr;
+    int st = check_dims(dims);
+    if (st != PA_OK) return st;
+    const pa_dims d = *dims;
+    if (d.num_seqs > 0 && (!h_cu || !h_seq)) return PA_ERR_NULL;
+    if (d.num_seqs == 0 && d.num_tokens != 0) return PA_ERR_SHAPE;
+    if (d.num_seqs > 0) {
+        if (h_cu[0] != 0 || h_cu[d.num_seqs] != d.num_tokens) return PA_ERR_SHAPE;
+        for (int i = 0; i < d.num_seqs; ++i) {
+            const int64_t L = (int64_t)h_cu[i + 1] - h_cu[i];
+            if (L < 0 || h_seq[i] < L) return PA_ERR_SHAPE;
+            if (L > 0 && cdiv(h_seq[i], pa::kBlockSize) > d.max_blocks_per_seq) return PA_ERR_SHAPE;
+        }
+    }
+
+    pa_plan *p = new (std::nothrow) pa_plan();
+    if (!p) return PA_ERR_CUDA;
+    p->dims = d;
+    p->group = d.num_q_heads / d.num_kv_heads;
+    p->num_sms = device >= 0 ? pa::device_sm_count(device) : 148;
+    const int Hkv = d.num_kv_heads;
+
+    std::vector<pa::DecodeRow> rows;
+    std::vector<pa::PrefillTile> tiles;
+    for (int i = 0; i < d.num_seqs; ++i) {
+        const int L = h_cu[i + 1] - h_cu[i];
+        const int n = h_seq[i];
+        if (L == 0) continue;
+        if (L <= pa::kDecodeMaxQLen || !pa::prefill_kernel_available()) {
+            for (int j = 0; j < L; ++j)
+                for (int g = 0; g < Hkv; ++g)
+                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow});
+        } else {
+            for (int q0 = 0; q0 < L; q0 += pa::kPrefillTileM) {
+                const int last = std::min(L, q0 + pa::kPrefillTileM) - 1;
+                const int kv_tiles = (int)cdiv(n - L + last + 1, pa::kPrefillTileN);
+                for (int h = 0; h < d.num_q_heads; ++h) tiles.push_back({i, q0, h, kv_tiles});
+            }
+            for (int j = 0; j < L; ++j) p->prefill_pairs += n - L + j + 1;
+        }
+    }
+    std::stable_sort(tiles.begin(), tiles.end(),
+                     [](const pa::PrefillTile &a, const pa::PrefillTile &b) {
+                         return a.n_kv_tiles > b.n_kv_tiles;
+                     });
+
+    // Cut the decode rows' blocks into equal runs.
+    const int64_t R = (int64_t)rows.size();
+    std::vector<int64_t> prefix(R + 1, 0);
+    for (int64_t r = 0; r < R; ++r) prefix[r + 1] = prefix[r] + cdiv(rows[r].n_keys, pa::kBlockSize);
+    const int64_t total = prefix[R];
+    int64_t P = 0;
+    if (total > 0) {
+        const int64_t max_units = (int64_t)p->num_sms * pa::decode_warps_per_sm(d.head_dim);
+        P = std::max<int64_t>(1, std::min(max_units, cdiv(total, kMinBlocksPerUnit)));
+    }
+    std::vector<pa::DecodeUnit> units(P + 1);
+    std::vector<int64_t> ustart(P + 1);
+    {
+        int64_t r = 0;
+        for (int64_t u = 0; u <= P; ++u) {
+            const int64_t f = P ? total * u / P : 0;
+            ustart[u] = f;
+            while (r < R && prefix[r + 1] <= f) ++r;  // row holding block f
+            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)])};
+        }
+        units[P] = {(int32_t)R, 0};
+    }
+    // Pieces: a row is split if its blocks span more than one unit.
+    std::vector<pa::CombineRow> combine;
+    int32_t piece_base = 0;
+    {
+        int64_t u = 0;
+        for (int64_t r = 0; r < R; ++r) {
+            while (u + 1 < P && ustart[u + 1] <= prefix[r]) ++u;  // unit of the first block
+            int64_t v = u;
+            while (v + 1 < P && ustart[v + 1] <= prefix[r + 1] - 1) ++v;  // unit of the last block
+            const int32_t count = (int32_t)(v - u + 1);
+            if (count > 1) {
+                rows[r].slot_base = piece_base - (int32_t)u;
+                combine.push_back({(int32_t)r, piece_base, count, 0});
+                piece_base += count;
+            }
+        }
+    }
+
+    p->num_units = (int32_t)P;
+    p->num_rows = (int32_t)R;
+    p->num_pieces = piece_base;
+    p->num_combine = (int32_t)combine.size();
+    p->decode_blocks = total;
+    p->num_tiles = (int32_t)tiles.size();
+
+    pa::WorkspaceLayout &w = p->ws;
+    size_t off = 0;
+    w.units = off;   off = align_up(off + sizeof(pa::DecodeUnit) * units.size(), pa::kWorkspaceAlign);
+    w.rows = off;    off = align_up(off + sizeof(pa::DecodeRow) * rows.size(), pa::kWorkspaceAlign);
+    w.combine = off; off = align_up(off + sizeof(pa::CombineRow) * combine.size(), pa::kWorkspaceAlign);
+    w.tiles = off;   off = align_up(off + sizeof(pa::PrefillTile) * tiles.size(), pa::kWorkspaceAlign);
+    w.table_bytes = off;
+    w.partial_o = off;
+    off = align_up(off + sizeof(float) * (size_t)piece_base * p->group * d.head_dim, pa::kWorkspaceAlign);
+    w.partial_ml = off;
+    off = align_up(off + sizeof(float) * 2 * (size_t)piece_base * p->group, pa::kWorkspaceAlign);
+    w.total = off;
+
+    try {
+        p->tables.assign(w.table_bytes, 0);
+    } catch (...) {
+        delete p;
+        return PA_ERR_CUDA;
+    }
+    std::memcpy(p->tables.data() + w.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
+    if (!rows.empty())
+        std::memcpy(p->tables.data() + w.rows, rows.data(), sizeof(pa::DecodeRow) * rows.size());
+    if (!combine.empty())
+        std::memcpy(p->tables.data() + w.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
+    if (!tiles.empty())
+        std::memcpy(p->tables.data() + w.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
+    *out = p;
+    return PA_OK;
+}
+
+extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
+    if (!p || !info) return PA_ERR_NULL;
+    info->num_sms = p->num_sms;
+    info->num_decode_rows = p->num_rows;
+    info->num_decode_units = p->num_units;
+    info->num_partials = p->num_pieces;
+    info->num_combine_rows = p->num_combine;
+    info->num_prefill_tiles = p->num_tiles;
+    info->decode_kv_blocks = p->decode_blocks;
+    info->prefill_causal_pairs = p->prefill_pairs;
+    info->table_bytes = p->ws.table_bytes;
+    info->workspace_bytes = p->ws.total;
+    return PA_OK;
+}
+
+extern "C" size_t pa_plan_workspace_bytes(const pa_plan *plan) { return plan ? plan->ws.total : 0; }
+
+extern "C" void pa_plan_destroy(pa_plan *plan) { delete plan; }

@@ -1,0 +1,92 @@
+// Internal layout of a pa_plan (host) and of the tables it copies into the
+// workspace (device).  Shared by plan.cpp and the CUDA sources; not part of
+// the public ABI.
+#pragma once
+#include <cstddef>
+#include <climits>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+constexpr int kBlockSize = 16;
+// Segments with q_len above this go to the tensor-core prefill kernel; the
+// others are handled as independent query rows by the split-KV decode kernel.
+constexpr int kDecodeMaxQLen = 16;
+constexpr int kPrefillTileM = 128;  // query rows per prefill tile
+constexpr int kPrefillTileN = 128;  // keys per prefill KV tile
+constexpr size_t kWorkspaceAlign = 256;
+// DecodeRow::slot_base of a row one warp covers entirely.  Split rows hold
+// piece_base - first_unit, which may be negative, so the marker lies below
+// every value that difference can take.
+constexpr int32_t kUnsplitRow = INT32_MIN;
+
+// One decode row: a query token and one kv head (the G query heads of that
+// kv head are computed together).  Row id r = token_row * Hkv + kv_head.
+struct DecodeRow {
+    int32_t token;      // flat token index t
+    int32_t seq;        // segment index i (block-table row)
+    int32_t n_keys;     // keys this query sees: p + 1
+    int32_t slot_base;  // kUnsplitRow: one warp covers the row and writes out
+                        // directly; else partial slot of unit u is slot_base + u
+};
+
+// A decode warp's work: flat (row, block) range [start, next unit's start).
+struct DecodeUnit {
+    int32_t row;
+    int32_t block;
+};
+
+// A row cut across several units: the combine step merges its partials.
+struct CombineRow {
+    int32_t row;
+    int32_t piece_base;
+    int32_t piece_count;
+    int32_t pad;
+};
+
+// One prefill tile: up to 128 consecutive queries of one segment, one query
+// head.
+struct PrefillTile {
+    int32_t seq;        // segment index
+    int32_t q_start;    // first query of the tile within the segment (j)
+    int32_t head;       // query head
+    int32_t n_kv_tiles; // 128-key tiles the tile reads (work estimate)
+};
+
+struct WorkspaceLayout {
+    size_t units = 0, rows = 0, combine = 0, tiles = 0;  // byte offsets
+    size_t table_bytes = 0;                              // bytes copied from the plan
+    size_t partial_o = 0, partial_ml = 0;                // scratch offsets
+    size_t total = 0;
+};
+
+}  // namespace pa
+
+struct pa_plan {
+    pa_dims dims{};
+    int num_sms = 148;
+    int group = 1;                       // Hq / Hkv
+    // decode part
+    int32_t num_units = 0;
+    int32_t num_rows = 0;
+    int32_t num_pieces = 0;
+    int32_t num_combine = 0;
+    int64_t decode_blocks = 0;           // sum over rows of ceil(n_keys / 16)
+    // prefill part
+    int32_t num_tiles = 0;
+    int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
+    pa::WorkspaceLayout ws;
+    std::vector<uint8_t> tables;         // image of [units | rows | combine | tiles]
+};
+
+namespace pa {
+// Decode warps a launch can keep resident per SM for a head dim.
+int decode_warps_per_sm(int head_dim);
+// SM count of a device (cached per process; 148 when it cannot be read).
+int device_sm_count(int device);
+// Whether long segments go to the tensor-core prefill kernel.
+bool prefill_kernel_available();
+}  // namespace pa

@@ -1,0 +1,266 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Cache writes must match bit for bit; attention (bf16 output converted to
+fp32) must be within max |err| 2e-2 and mean |err| 2e-3 of the fp64 oracle.
+Small cases compare every output row; the full-size workloads run exactly as
+bench.py launches them and compare sampled rows, which the oracle computes
+one by one on the host from the same (pre-write) pool.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import paged_kv_attention_token_b200 as pa
+import workloads as W
+from tests.parity import assert_parity, errors
+
+pytestmark = pytest.mark.gpu
+
+
+def dims_for(lay):
+    return pa.Dims(lay.num_tokens, lay.num_seqs, lay.num_q_heads, lay.num_kv_heads,
+                   lay.head_dim, lay.num_blocks, lay.max_blocks_per_seq, 16)
+
+
+def run_step(batch):
+    """Scatter then attention on the GPU, as one forward step does."""
+    lay = batch.layout
+    kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
+    bt, cu, sl, slots = batch.device_ints("cuda")
+    pa.reshape_and_cache(batch.k, batch.v, slots, kc, vc)
+    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay))
+    ws = pa.workspace_for(plan)
+    out = torch.full_like(batch.q, float("nan"))
+    pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws)
+    torch.cuda.synchronize()
+    return kc, vc, out, plan
+
+
+def oracle_subset(batch, seq_ids, queries=None):
+    """Oracle output for the given segments (all their query rows, or only
+    the listed query offsets per segment), from the pre-write pool."""
+    hs = W.host_subset(batch, seq_ids)
+    kc, vc = hs.k_cache.copy(), hs.v_cache.copy()
+    O.reshape_and_cache(hs.k, hs.v, hs.slot_mapping, kc, vc)
+    Hq = batch.layout.num_q_heads
+    if queries is None:
+        out = O.attention_varlen(hs.q, kc, vc, hs.block_tables, hs.cu_seqlens_q, hs.seq_lens, batch.scale)
+        return hs.token_index, out
+    toks = []
+    for r, s in enumerate(hs.seq_index):
+        L = hs.cu_seqlens_q[r + 1] - hs.cu_seqlens_q[r]
+        for j in queries.get(int(s), range(L)):
+            if 0 <= j < L:
+                toks.append(hs.cu_seqlens_q[r] + j)
+    toks = np.array(sorted(set(toks)), dtype=np.int64)
+    rows = (toks[:, None] * Hq + np.arange(Hq)[None, :]).reshape(-1)
+    out = O.attention_varlen(hs.q, kc, vc, hs.block_tables, hs.cu_seqlens_q, hs.seq_lens,
+                             batch.scale, rows=rows).reshape(len(toks), Hq, -1)
+    return hs.token_index[toks], out
+
+
+def gpu_rows(out, tokens):
+    return out[torch.from_numpy(np.asarray(tokens)).cuda()].float().cpu().numpy()
+
+
+# --------------------------------------------------------------------------
+# reshape_and_cache: bit-exact
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_scatter_bit_exact(cuda_lib, name):
+    lay = W.layout(name)
+    b = W.make_batch(lay, device="cuda")
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    _, _, _, slots = b.device_ints("cuda")
+    pa.reshape_and_cache(b.k, b.v, slots, kc, vc)
+    torch.cuda.synchronize()
+    # blocks holding a written slot: compare with the oracle's writes
+    touched = np.unique(lay.slot_mapping // 16)
+    tt = torch.from_numpy(touched).cuda()
+    pre_k, pre_v = W.bf16_bits(b.k_cache[tt]).copy(), W.bf16_bits(b.v_cache[tt]).copy()
+    remap = {int(x): i for i, x in enumerate(touched)}
+    s2 = np.array([remap[int(s) // 16] * 16 + int(s) % 16 for s in lay.slot_mapping], np.int64)
+    O.reshape_and_cache(W.bf16_bits(b.k), W.bf16_bits(b.v), s2, pre_k, pre_v)
+    assert np.array_equal(W.bf16_bits(kc[tt]), pre_k)
+    assert np.array_equal(W.bf16_bits(vc[tt]), pre_v)
+    # every other block unchanged, bit for bit
+    keep = torch.ones(lay.num_blocks, dtype=torch.bool, device="cuda")
+    keep[tt] = False
+    assert torch.equal(kc[keep].view(torch.int16), b.k_cache[keep].view(torch.int16))
+    assert torch.equal(vc[keep].view(torch.int16), b.v_cache[keep].view(torch.int16))
+
+
+def test_scatter_negative_slots_skip(cuda_lib):
+    lay = W.layout("tiny_mixed")
+    b = W.make_batch(lay, device="cuda")
+    kc = b.k_cache.clone()
+    vc = b.v_cache.clone()
+    slots = torch.from_numpy(lay.slot_mapping).cuda()
+    slots[::2] = -1
+    pa.reshape_and_cache(b.k, b.v, slots, kc, vc)
+    pre_k, pre_v = W.bf16_bits(b.k_cache).copy(), W.bf16_bits(b.v_cache).copy()
+    O.reshape_and_cache(W.bf16_bits(b.k), W.bf16_bits(b.v), slots.cpu().numpy(), pre_k, pre_v)
+    assert np.array_equal(W.bf16_bits(kc), pre_k) and np.array_equal(W.bf16_bits(vc), pre_v)
+
+
+# --------------------------------------------------------------------------
+# attention, every row
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_tiny_mixed_all_rows(cuda_lib, q_gain):
+    lay = W.layout("tiny_mixed")
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, _ = run_step(b)
+    tok, want = oracle_subset(b, range(lay.num_seqs))
+    assert_parity(gpu_rows(out, tok), want, f"tiny_mixed q_gain={q_gain}")
+
+
+CUSTOM = [
+    # (q_lens, seq_lens, Hq, Hkv, D)
+    ([1, 1, 1, 1, 1, 1], [1, 15, 16, 17, 32, 33], 8, 1, 64),          # block edges, seq 1
+    ([1, 1, 1, 0, 3], [2000, 1999, 777, 40, 3], 32, 4, 64),           # long rows split across warps
+    ([1, 5, 1, 2], [1500, 37, 2100, 16], 32, 4, 128),
+    ([1, 1, 7, 1], [900, 4100, 33, 64], 12, 2, 128),                   # G = 6: padded heads
+    ([1, 1, 2], [300, 1030, 45], 16, 1, 128),                          # G = 16: two n-tiles
+    ([1, 3, 1], [513, 30, 257], 32, 2, 64),                            # G = 16 at D = 64
+    ([1, 1, 1], [129, 1025, 48], 4, 4, 128),                           # G = 1 (multi-head)
+    ([40, 1, 17], [40, 90, 100], 4, 2, 64),                            # prefill rows
+]
+
+
+@pytest.mark.parametrize("case", range(len(CUSTOM)))
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_custom_shapes_all_rows(cuda_lib, case, q_gain):
+    q_lens, seq_lens, Hq, Hkv, D = CUSTOM[case]
+    nb = sum(-(-s // 16) for s in seq_lens) + 64
+    lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, nb, seed=100 + case)
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, plan = run_step(b)
+    tok, want = oracle_subset(b, range(lay.num_seqs))
+    assert_parity(gpu_rows(out, tok), want, f"case {case} q_gain={q_gain} plan={plan.info()}")
+
+
+def test_split_rows_are_exercised(cuda_lib):
+    q_lens, seq_lens, Hq, Hkv, D = CUSTOM[1]
+    lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, 600, seed=101)
+    info = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay)).info()
+    assert info["num_combine_rows"] > 0 and info["num_partials"] > 2 * info["num_combine_rows"]
+
+
+# --------------------------------------------------------------------------
+# attention at full size, launched as bench.py launches it
+# --------------------------------------------------------------------------
+
+def _sample_seqs(lay, k, seed):
+    rng = np.random.default_rng(seed)
+    order = np.argsort(lay.seq_lens)
+    pick = {int(order[0]), int(order[-1])}              # shortest and longest
+    pick |= set(int(x) for x in rng.choice(lay.num_seqs, size=min(k, lay.num_seqs), replace=False))
+    return sorted(pick)
+
+
+@pytest.mark.parametrize("name,q_gain", [("decode_tinyllama_b64", 1.0), ("decode_tinyllama_b64", 8.0),
+                                         ("decode_llama3_8b_b256", 1.0),
+                                         ("prefix_llama3_70b_b128", 1.0)])
+def test_full_size_decode_sampled(cuda_lib, name, q_gain):
+    lay = W.layout(name)
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, _ = run_step(b)
+    assert not torch.isnan(out).any()
+    seqs = _sample_seqs(lay, 10, 7)
+    tok, want = oracle_subset(b, seqs)
+    assert_parity(gpu_rows(out, tok), want, name)
+
+
+@pytest.mark.slow
+def test_full_size_mixed_sampled(cuda_lib):
+    lay = W.layout("mixed_qwen25_1p5b_t8192")
+    b = W.make_batch(lay, device="cuda")
+    _, _, out, _ = run_step(b)
+    assert not torch.isnan(out).any()
+    S = lay.num_seqs
+    prefill = [S - 4, S - 3, S - 2, S - 1]
+    rng = np.random.default_rng(3)
+    decodes = sorted(int(x) for x in rng.choice(S - 4, size=6, replace=False))
+    qs = {s: [0, 1, 15, 16, 127, 128, 129, 500, 1023, 1024, 1535, 2047, 2431] for s in prefill}
+    tok, want = oracle_subset(b, prefill + decodes, queries=qs)
+    assert_parity(gpu_rows(out, tok), want, "mixed")
+
+
+def test_deterministic(cuda_lib):
+    lay = W.layout("decode_tinyllama_b64")
+    b = W.make_batch(lay, device="cuda")
+    _, _, o1, _ = run_step(b)
+    _, _, o2, _ = run_step(b)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def test_plan_reused_across_calls_and_streams(cuda_lib):
+    lay = W.layout("decode_tinyllama_b64")
+    b = W.make_batch(lay, device="cuda")
+    kc, vc, ref, plan = run_step(b)
+    bt, cu, sl, _ = b.device_ints("cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ws = pa.workspace_for(plan)
+        out = torch.empty_like(b.q)
+        for _ in range(3):
+            pa.attention_varlen(b.q, kc, vc, bt, cu, sl, b.scale, out, plan, ws, stream=s)
+    s.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+# --------------------------------------------------------------------------
+# validation and binding errors
+# --------------------------------------------------------------------------
+
+def test_validate_inputs(cuda_lib):
+    lay = W.layout("tiny_mixed")
+    b = W.make_batch(lay, device="cuda")
+    bt, cu, sl, slots = b.device_ints("cuda")
+    d = dims_for(lay)
+    assert pa.validate_inputs(slots, bt, cu, sl, d) == pa.PA_OK
+    bad = slots.clone(); bad[0] = lay.num_blocks * 16
+    assert pa.validate_inputs(bad, bt, cu, sl, d) == pa.PA_ERR_BOUNDS
+    dup = slots.clone(); dup[1] = dup[0]
+    assert pa.validate_inputs(dup, bt, cu, sl, d) == pa.PA_ERR_BOUNDS
+    bt2 = bt.clone(); bt2[0, 0] = lay.num_blocks
+    assert pa.validate_inputs(slots, bt2, cu, sl, d) == pa.PA_ERR_BOUNDS
+    sl2 = sl.clone(); sl2[2] = 3                       # q_len 6 > seq_len 3
+    assert pa.validate_inputs(slots, bt, cu, sl2, d) == pa.PA_ERR_BOUNDS
+    # block-table padding is never checked (it is never read)
+    bt3 = bt.clone(); bt3[2, 1:] = -5
+    assert pa.validate_inputs(slots, bt3, cu, sl, d) == pa.PA_OK
+
+
+def test_binding_rejects_wrong_dtypes(cuda_lib):
+    lay = W.layout("tiny_mixed")
+    b = W.make_batch(lay, device="cuda")
+    bt, cu, sl, slots = b.device_ints("cuda")
+    with pytest.raises(pa.PaError):
+        pa.reshape_and_cache(b.k.float(), b.v, slots, b.k_cache, b.v_cache)
+    with pytest.raises(pa.PaError):
+        pa.reshape_and_cache(b.k, b.v, slots.int(), b.k_cache, b.v_cache)
+    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay))
+    ws = pa.workspace_for(plan)
+    with pytest.raises(pa.PaError):
+        pa.attention_varlen(b.q, b.k_cache, b.v_cache, bt.long(), cu, sl, b.scale,
+                            torch.empty_like(b.q), plan, ws)
+
+
+def test_traced_call_matches_and_times_each_kernel(cuda_lib):
+    lay = W.layout("decode_tinyllama_b64")
+    b = W.make_batch(lay, device="cuda")
+    kc, vc, ref, plan = run_step(b)
+    bt, cu, sl, _ = b.device_ints("cuda")
+    ws = pa.workspace_for(plan)
+    out = torch.empty_like(b.q)
+    tr = pa.Trace()
+    pa.attention_varlen(b.q, kc, vc, bt, cu, sl, b.scale, out, plan, ws, trace=tr)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    t = tr.elapsed_ms()
+    assert t["decode"] > 0 and t["combine"] >= 0 and t["total"] >= t["decode"]
