@@ -12,15 +12,17 @@ attention shapes only; no weights).  Default workload: 64 decodes with the
 TinyLlama-1.1B attention shape.
 
 Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier and
-torch.cuda.synchronize() on both sides.  L2 is flushed (a 512 MiB write)
+torch.cuda.synchronize() on both sides.  L2 is flushed (a 1 GiB write)
 before every step and each step's device time is taken with CUDA events on
 the launching stream, excluding the flush; the host plan for a step is built
-while the flush runs.  Multi-GPU (torchrun): every rank runs its own batch of
+and its kernels queued while the flush runs, so the events see device time
+rather than host launch overhead.  Multi-GPU (torchrun): every rank runs its own batch of
 the same shape (weak scaling, no collective on the data path); the reported
 time is the max over ranks.
 
-The JSON line adds: roofline (dominant kernel, timed live with CUDA events
-around it), e2e (same metric through the public API with host buffers: H2D of
+The JSON line adds: roofline (dominant kernel, timed in the same run with
+CUDA events around it on its stream, in a second pass of K identical steps,
+since event records cost GPU time of their own), e2e (same metric through the public API with host buffers: H2D of
 the step's inputs and D2H of its output inside the timed region), the CPU
 oracle as a reported baseline, SM clocks sampled during the timed region, and
 the number of library kernels launched.
@@ -50,7 +52,7 @@ import workloads as W  # noqa: E402
 METRIC = "paged-attn decode KV GB/s (% of HBM peak); mixed-batch attn tokens/s, % roofline"
 DEFAULT_WORKLOAD = "decode_tinyllama_b64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FLUSH_BYTES = 512 << 20
+FLUSH_BYTES = 1 << 30
 
 
 # ---------------------------------------------------------------------------
@@ -314,10 +316,15 @@ def run_ours(args):
     launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + \
         (1 if info["num_combine_rows"] else 0) + (1 if info["num_prefill_tiles"] else 0)
 
+    # two plans rebuilt in turn, as an engine keeps them across steps
+    plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local), pa.Plan(h_cu, h_sl, dims, device=local)]
+    step_no = [0]
+
     def one_step(trace=None, ev=None):
         flush.fill_(1)
         t0 = time.perf_counter()
-        plan = pa.Plan(h_cu, h_sl, dims, device=local)
+        plan = plan_pool[step_no[0] % 2].rebuild(h_cu, h_sl, dims)
+        step_no[0] += 1
         plan_s = time.perf_counter() - t0
         if ev is not None:
             ev[0].record(stream)
@@ -332,7 +339,6 @@ def run_ours(args):
         one_step()
     torch.cuda.synchronize(dev)
 
-    traces = [pa.Trace() for _ in range(args.steps)]
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     clocks = ClockSampler(dev)
@@ -343,7 +349,7 @@ def run_ours(args):
     plans, plan_times = [], []
     wall0 = time.perf_counter()
     for i in range(args.steps):
-        plan, plan_s = one_step(traces[i], evs[i])
+        plan, plan_s = one_step(None, evs[i])
         plans.append(plan)
         plan_times.append(plan_s)
     torch.cuda.synchronize(dev)
@@ -352,7 +358,6 @@ def run_ours(args):
         dist.barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    stages = [t.elapsed_ms() for t in traces]
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if dist is not None:
@@ -367,11 +372,24 @@ def run_ours(args):
         unit = "tokens/s"
         value = world * lay.num_tokens * args.steps / (max_total_ms * 1e-3)
 
-    # roofline of the dominant kernel: the split-KV decode kernel
+    # Roofline of the dominant kernel (the split-KV decode kernel).  Event
+    # records cost GPU time, so the kernel is timed in a second pass of K
+    # steps, identical to the timed ones, with events around that kernel only
+    # (and, in a third pass, around the other stages of the call).
     peaks, peak_kind = load_peaks()
-    dec_ms = statistics.mean(s["decode"] for s in stages)
-    comb_ms = statistics.mean(s["combine"] for s in stages)
-    copy_ms = statistics.mean(s["table_copy"] for s in stages)
+
+    def traced_pass(stages):
+        trs = [pa.Trace(stages=stages) for _ in range(args.steps)]
+        for i in range(args.steps):
+            one_step(trs[i], None)
+        torch.cuda.synchronize(dev)
+        return [t.elapsed_ms() for t in trs]
+
+    dec_ms = statistics.mean(s["decode"] for s in traced_pass(("decode",)))
+    other = traced_pass(("table_copy", "combine", "prefill"))
+    comb_ms = statistics.mean(s["combine"] for s in other)
+    copy_ms = statistics.mean(s["table_copy"] for s in other)
+    prefill_ms = statistics.mean(s["prefill"] for s in other)
     dec_bytes = acct["kv"] + acct["qo"] + acct["meta"]
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     src_hash = kernel_source_hash(["decode.cu", "common.cuh", "kernels.h", "plan.h"])
@@ -398,7 +416,7 @@ def run_ours(args):
             e0.record(stream)
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
-            plan = pa.Plan(h_cu, h_sl, dims, device=local)
+            plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims)
             pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)
             pa.attention_varlen(dev_in["q"], kc, vc, dev_in["bt"], dev_in["cu"], dev_in["sl"],
                                 batch.scale, out, plan, ws, stream=stream)
@@ -434,10 +452,11 @@ def run_ours(args):
             "config": {"workload": args.workload, "shape": lay.description,
                        "bytes_per_step": acct["total"], "kv_bytes_per_step": acct["kv"],
                        "tokens_per_step": lay.num_tokens,
-                       "l2": "flushed before every timed step (512 MiB write, outside the events)",
+                       "l2": "flushed before every timed step (1 GiB write, outside the events)",
                        "plan_us_host": 1e6 * statistics.median(plan_times),
                        "stages_ms": {"table_copy": copy_ms, "decode": dec_ms, "combine": comb_ms,
-                                     "prefill": statistics.mean(s["prefill"] for s in stages)},
+                                     "prefill": prefill_ms,
+                                     "note": "separate traced passes; event records add GPU time"},
                        "parallelism": f"replicas x{world} (weak: one batch per GPU)",
                        "wall_s_timed_region": wall},
             "roofline": roofline,
@@ -456,7 +475,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -110,9 +110,19 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  *   dims            host; T, S, Hq, Hkv, D, B are used
  *   device          CUDA device ordinal the plan is sized for (its SM count
  *                   is read once per process and cached; -1 = assume 148 SMs)
- *   out             receives a new plan owned by the caller; free it with
- *                   pa_plan_destroy.  A plan is immutable and may be reused
- *                   for every layer of a step, and by several streams.
+ *   out             in/out.  If *out is NULL a new plan is created and
+ *                   stored there; the caller owns it and frees it with
+ *                   pa_plan_destroy.  If *out holds a plan from an earlier
+ *                   call (same device), that plan is rebuilt in place and its
+ *                   host buffers are reused, so that a caller rebuilding one
+ *                   plan per step allocates nothing after the first step.
+ *                   The plan's tables live in page-locked host memory and are
+ *                   copied into the workspace by every attention call that
+ *                   uses the plan; rebuilding or destroying a plan first waits
+ *                   until the most recent such copy has executed.  A plan may
+ *                   serve every layer of a step and several streams.
+ * On error a plan passed in *out is left unusable for attention calls until
+ * it is rebuilt successfully; it must still be destroyed.
  * Errors: PA_ERR_NULL, PA_ERR_SHAPE (cu_seqlens not starting at 0, not
  * non-decreasing or not ending at T; q_len > seq_len), PA_ERR_UNSUPPORTED.
  */
@@ -139,9 +149,9 @@ int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
  * (0 for a NULL plan).  256-byte alignment of the workspace is required. */
 size_t pa_plan_workspace_bytes(const pa_plan *plan);
 
-/* Frees a plan (NULL is allowed).  Work already queued that used the plan is
- * not affected: the plan's tables are copied into the workspace when the
- * call is queued. */
+/* Frees a plan (NULL is allowed), after waiting until the table copy of the
+ * most recent attention call that used it has executed.  Work queued with it
+ * is not affected. */
 void pa_plan_destroy(pa_plan *plan);
 
 /*

@@ -169,21 +169,30 @@ def _host_i32(a, name):
 
 
 class Plan:
-    """Work partition for one step (pa_plan_build); reusable for every layer."""
+    """Work partition for one step (pa_plan_build); reusable for every layer.
+
+    The plan must stay alive until the GPU work queued with it has completed
+    (like every other input).  ``rebuild`` re-partitions for the next step in
+    place, reusing the plan's page-locked buffer."""
 
     def __init__(self, cu_seqlens_q, seq_lens, dims: Dims, device: int | None = None):
         lib = load_library()
         self._lib = lib
+        if device is None:
+            device = torch.cuda.current_device() if torch.cuda.is_available() else -1
+        self.device = int(device)
+        self._h = ctypes.c_void_p()
+        self.rebuild(cu_seqlens_q, seq_lens, dims)
+
+    def rebuild(self, cu_seqlens_q, seq_lens, dims: Dims):
         self._cu = _host_i32(cu_seqlens_q, "cu_seqlens_q")
         self._sl = _host_i32(seq_lens, "seq_lens")
         self.dims = Dims(*[getattr(dims, n) for n, _ in Dims._fields_])
-        if device is None:
-            device = torch.cuda.current_device() if torch.cuda.is_available() else -1
-        h = ctypes.c_void_p()
-        _check(lib.pa_plan_build(self._cu.ctypes.data_as(ctypes.c_void_p),
-                                 self._sl.ctypes.data_as(ctypes.c_void_p), ctypes.byref(self.dims),
-                                 int(device), ctypes.byref(h)), "pa_plan_build")
-        self._h = h
+        _check(self._lib.pa_plan_build(self._cu.ctypes.data_as(ctypes.c_void_p),
+                                       self._sl.ctypes.data_as(ctypes.c_void_p),
+                                       ctypes.byref(self.dims), self.device, ctypes.byref(self._h)),
+               "pa_plan_build")
+        return self
 
     @property
     def handle(self):
@@ -220,27 +229,30 @@ class Trace(ctypes.Structure):
     """Events recorded around the kernels of one attention call (pa_trace)."""
     _fields_ = [("events", ctypes.c_void_p * 6)]
 
-    STAGES = ("table_copy", "decode", "combine", "gap", "prefill")
+    MARKS = {"table_copy": (0, 1), "decode": (1, 2), "combine": (2, 3), "prefill": (4, 5)}
 
-    def __init__(self):
+    def __init__(self, stages=("table_copy", "decode", "combine", "prefill")):
+        """Record only the marks the named stages need (each record costs a
+        couple of microseconds of GPU time)."""
         super().__init__()
-        self.torch_events = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-        for i, e in enumerate(self.torch_events):
-            self.events[i] = ctypes.c_void_p(e.cuda_event)
+        self.stages = tuple(stages)
+        used = sorted({i for st in self.stages for i in self.MARKS[st]})
+        self.torch_events = {i: torch.cuda.Event(enable_timing=True) for i in used}
 
     def arm(self, stream):
         # torch only reports elapsed times of events it has recorded itself;
         # record them once here, the library records them again at its marks
         # (the latest record on the stream sets an event's timestamp).
-        for e in self.torch_events:
+        # torch creates the CUDA event on its first record, so the handles
+        # are taken only after that
+        for i, e in self.torch_events.items():
             e.record(stream)
+            self.events[i] = ctypes.c_void_p(e.cuda_event)
 
     def elapsed_ms(self) -> dict:
         """Per-stage times (ms) once the stream has reached the last event."""
         ev = self.torch_events
-        return {"table_copy": ev[0].elapsed_time(ev[1]), "decode": ev[1].elapsed_time(ev[2]),
-                "combine": ev[2].elapsed_time(ev[3]), "prefill": ev[4].elapsed_time(ev[5]),
-                "total": ev[0].elapsed_time(ev[5])}
+        return {st: ev[self.MARKS[st][0]].elapsed_time(ev[self.MARKS[st][1]]) for st in self.stages}
 
 
 def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale,

@@ -140,10 +140,13 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
     if (w.table_bytes > 0) {
-        // Pageable source: the runtime stages it before returning, so the plan
-        // may be destroyed or rebuilt as soon as this call returns.
-        if (cudaMemcpyAsync(ws, plan->tables.data(), w.table_bytes, cudaMemcpyHostToDevice,
-                            stream) != cudaSuccess)
+        // Page-locked source: the copy runs in stream order without blocking
+        // the host; the plan's event marks when its buffer may be reused.
+        if (cudaMemcpyAsync(ws, plan->tables, w.table_bytes, cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess)
+            return PA_ERR_CUDA;
+        if (plan->upload_event &&
+            cudaEventRecord(static_cast<cudaEvent_t>(plan->upload_event), stream) != cudaSuccess)
             return PA_ERR_CUDA;
     }
     const float scale_log2 = scale * kLog2e;

@@ -14,8 +14,11 @@
 // Prefill side (longer segments): 128-query tiles per query head, ordered by
 // the number of 128-key tiles they read, longest first.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <new>
+
+#include <cuda_runtime.h>
 
 #include "plan.h"
 
@@ -28,6 +31,62 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Fewest KV blocks one decode warp is given, so that per-warp fixed costs
 // (loading q, the final write) stay small against the streaming.
 constexpr int64_t kMinBlocksPerUnit = 4;
+
+// Waits until the last table copy queued from this plan has executed.
+void wait_upload(const pa_plan *p) {
+    if (p->upload_event) cudaEventSynchronize(static_cast<cudaEvent_t>(p->upload_event));
+}
+
+void free_tables(pa_plan *p) {
+    if (!p->tables) return;
+    if (p->tables_pinned)
+        cudaFreeHost(p->tables);
+    else
+        std::free(p->tables);
+    p->tables = nullptr;
+    p->tables_capacity = 0;
+    p->tables_pinned = false;
+}
+
+// Host buffer of at least `bytes` for the plan tables: page-locked when the
+// plan has a device, ordinary memory otherwise (host-only use, tests).
+bool reserve_tables(pa_plan *p, size_t bytes) {
+    if (p->tables && p->tables_capacity >= bytes) return true;
+    free_tables(p);
+    const size_t cap = std::max<size_t>(bytes, 4096);
+    if (p->device >= 0) {
+        int prev = -1;
+        cudaGetDevice(&prev);
+        if (prev != p->device) cudaSetDevice(p->device);
+        void *h = nullptr;
+        if (cudaHostAlloc(&h, cap, cudaHostAllocPortable) == cudaSuccess) {
+            p->tables = static_cast<uint8_t *>(h);
+            p->tables_pinned = true;
+        } else {
+            cudaGetLastError();
+        }
+        if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
+    }
+    if (!p->tables) {
+        p->tables = static_cast<uint8_t *>(std::malloc(cap));
+        if (!p->tables) return false;
+    }
+    p->tables_capacity = cap;
+    return true;
+}
+
+void create_event(pa_plan *p) {
+    if (p->upload_event || p->device < 0) return;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != p->device) cudaSetDevice(p->device);
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess)
+        p->upload_event = e;
+    else
+        cudaGetLastError();
+    if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
+}
 
 int check_dims(const pa_dims *d) {
     if (!d) return PA_ERR_NULL;
@@ -50,7 +109,6 @@ int decode_warps_per_sm(int head_dim) { return head_dim <= 64 ? 16 : 8; }
 extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa_dims *dims,
                              int device, pa_plan **out) {
     if (!out) return PA_ERR_NULL;
-    *out = nullptr;
     int st = check_dims(dims);
     if (st != PA_OK) return st;
     const pa_dims d = *dims;
@@ -65,11 +123,20 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
         }
     }
 
-    pa_plan *p = new (std::nothrow) pa_plan();
-    if (!p) return PA_ERR_CUDA;
+    pa_plan *p = *out;
+    const bool fresh = (p == nullptr);
+    if (fresh) {
+        p = new (std::nothrow) pa_plan();
+        if (!p) return PA_ERR_CUDA;
+        p->device = device;
+        create_event(p);
+    } else if (p->device != device) {
+        return PA_ERR_PLAN;
+    }
     p->dims = d;
     p->group = d.num_q_heads / d.num_kv_heads;
     p->num_sms = device >= 0 ? pa::device_sm_count(device) : 148;
+    p->prefill_pairs = 0;
     const int Hkv = d.num_kv_heads;
 
     std::vector<pa::DecodeRow> rows;
@@ -156,19 +223,19 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     off = align_up(off + sizeof(float) * 2 * (size_t)piece_base * p->group, pa::kWorkspaceAlign);
     w.total = off;
 
-    try {
-        p->tables.assign(w.table_bytes, 0);
-    } catch (...) {
-        delete p;
+    wait_upload(p);  // the previous build's tables may still be in a queued copy
+    if (!reserve_tables(p, w.table_bytes)) {
+        if (fresh) pa_plan_destroy(p);
         return PA_ERR_CUDA;
     }
-    std::memcpy(p->tables.data() + w.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
+    std::memset(p->tables, 0, w.table_bytes);
+    std::memcpy(p->tables + w.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
     if (!rows.empty())
-        std::memcpy(p->tables.data() + w.rows, rows.data(), sizeof(pa::DecodeRow) * rows.size());
+        std::memcpy(p->tables + w.rows, rows.data(), sizeof(pa::DecodeRow) * rows.size());
     if (!combine.empty())
-        std::memcpy(p->tables.data() + w.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
+        std::memcpy(p->tables + w.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
     if (!tiles.empty())
-        std::memcpy(p->tables.data() + w.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
+        std::memcpy(p->tables + w.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
     *out = p;
     return PA_OK;
 }
@@ -190,4 +257,10 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
 
 extern "C" size_t pa_plan_workspace_bytes(const pa_plan *plan) { return plan ? plan->ws.total : 0; }
 
-extern "C" void pa_plan_destroy(pa_plan *plan) { delete plan; }
+extern "C" void pa_plan_destroy(pa_plan *plan) {
+    if (!plan) return;
+    wait_upload(plan);
+    free_tables(plan);
+    if (plan->upload_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->upload_event));
+    delete plan;
+}

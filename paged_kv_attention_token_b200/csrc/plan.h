@@ -79,7 +79,15 @@ struct pa_plan {
     int32_t num_tiles = 0;
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::WorkspaceLayout ws;
-    std::vector<uint8_t> tables;         // image of [units | rows | combine | tiles]
+    // Image of [units | rows | combine | tiles], copied into the workspace by
+    // every attention call.  Page-locked when a device is present, so that the
+    // copy is truly asynchronous; the event is recorded after each copy, and a
+    // rebuild or destroy waits on it before touching the buffer.
+    uint8_t *tables = nullptr;
+    size_t tables_capacity = 0;
+    bool tables_pinned = false;
+    void *upload_event = nullptr;        // cudaEvent_t, or null without a device
+    int device = -1;
 };
 
 namespace pa {

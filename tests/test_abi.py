@@ -82,6 +82,26 @@ def test_plan_invariants(lib, name):
     assert plan.workspace_bytes == info["workspace_bytes"]
 
 
+def test_plan_rebuild_in_place(lib):
+    a = W.layout("decode_tinyllama_b64")
+    b = W.layout("tiny_mixed")
+    plan = pa.Plan(a.cu_seqlens_q, a.seq_lens, dims_for(a), device=-1)
+    h0 = plan.handle.value
+    ia = plan.info()
+    plan.rebuild(b.cu_seqlens_q, b.seq_lens, dims_for(b))
+    assert plan.handle.value == h0
+    ib = plan.info()
+    assert ib == pa.Plan(b.cu_seqlens_q, b.seq_lens, dims_for(b), device=-1).info()
+    plan.rebuild(a.cu_seqlens_q, a.seq_lens, dims_for(a))
+    assert plan.info() == ia
+    # a plan cannot move to another device
+    h = plan.handle
+    d = dims_for(a)
+    assert lib.pa_plan_build(a.cu_seqlens_q.ctypes.data_as(ctypes.c_void_p),
+                             a.seq_lens.ctypes.data_as(ctypes.c_void_p), ctypes.byref(d), 0,
+                             ctypes.byref(h)) == pa.PA_ERR_PLAN
+
+
 def test_plan_is_deterministic(lib):
     lay = W.layout("decode_llama3_8b_b256")
     a = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay), device=-1).info()
@@ -96,14 +116,17 @@ def _status(fn, *args):
 def test_plan_rejects_bad_arguments(lib):
     lay = W.layout("tiny_mixed")
     cu, sl = lay.cu_seqlens_q.copy(), lay.seq_lens.copy()
-    h = ctypes.c_void_p()
 
     def build(cu, sl, d):
-        return lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p),
-                                 ctypes.byref(d), -1, ctypes.byref(h))
+        h = ctypes.c_void_p()          # NULL: ask for a new plan
+        st = lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p),
+                               ctypes.byref(d), -1, ctypes.byref(h))
+        assert st == pa.PA_OK or not h.value
+        lib.pa_plan_destroy(h)
+        return st
 
+    h = ctypes.c_void_p()
     assert build(cu, sl, dims_for(lay)) == pa.PA_OK
-    lib.pa_plan_destroy(h)
     bad = cu.copy(); bad[-1] += 1
     assert build(bad, sl, dims_for(lay)) == pa.PA_ERR_SHAPE          # does not end at T
     bad = cu.copy(); bad[1], bad[2] = bad[2], bad[1]
