@@ -64,7 +64,9 @@ typedef enum {
     PA_ERR_WORKSPACE = -6,   /* workspace NULL or smaller than the plan needs */
     PA_ERR_BOUNDS = -7,      /* pa_validate_inputs found a precondition violated */
     PA_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
-    PA_ERR_PLAN = -9         /* the plan does not match the dims of the call */
+    PA_ERR_PLAN = -9,        /* the plan does not match the dims of the call */
+    PA_ERR_TOO_LARGE = -10   /* the call needs more scratch than the no-alloc
+                                entry point's fixed array holds */
 } pa_status;
 
 /* Sizes of one call.  block_size must be 16. */
@@ -224,6 +226,41 @@ int pa_validate_inputs(const int64_t *d_slot_mapping, const int32_t *d_block_tab
                        const int32_t *d_cu_seqlens_q, const int32_t *d_seq_lens,
                        const pa_dims *dims, void *d_scratch, size_t scratch_bytes,
                        void *stream);
+
+/*
+ * pa_attention_varlen_noalloc — the same computation as pa_attention_varlen,
+ * for callers that cannot allocate device memory.  The pages have no
+ * counterpart of this call: it exists for callers such as an engine that has
+ * given nearly all GPU memory to its KV pool and keeps no allocator in its
+ * step loop, a host or plugin interface that hands an op only its inputs,
+ * outputs and a stream, or a loop that must avoid the device-wide stalls a
+ * cudaMalloc/cudaFree pair can cause.
+ *
+ * Instead of a caller workspace it uses one fixed array of
+ * pa_noalloc_scratch_bytes() (16 MiB) in the library's device memory.  Every
+ * GPU that loads libpa.so holds that array until the process exits.  The call
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - Arguments and results are those of pa_attention_varlen, minus
+ *     d_workspace / workspace_bytes.
+ *   - A plan whose pa_plan_workspace_bytes exceeds the array is rejected with
+ *     PA_ERR_TOO_LARGE before any work is queued.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's device address with cudaGetSymbolAddress and caches it; make
+ *     that first call before any stream capture.  A failed lookup returns
+ *     PA_ERR_CUDA.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents.  Nothing in it needs to start at zero: every call first
+ *     copies its plan's tables over the front of it and writes each partial
+ *     result before reading it.  Calls whose GPU work overlaps in time (two
+ *     streams, or two threads' streams) race on the array and give undefined
+ *     results; order them, or use pa_attention_varlen with separate
+ *     workspaces.
+ */
+size_t pa_noalloc_scratch_bytes(void);
+int pa_attention_varlen_noalloc(const void *d_q, const void *d_k_cache, const void *d_v_cache,
+                                const int32_t *d_block_tables, const int32_t *d_cu_seqlens_q,
+                                const int32_t *d_seq_lens, float scale, void *d_out,
+                                const pa_dims *dims, const pa_plan *plan, void *stream);
 
 /* Static text for a status code. */
 const char *pa_status_string(int status);

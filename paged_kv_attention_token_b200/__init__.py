@@ -25,10 +25,12 @@ __all__ = ["load_library", "library_path", "PaError", "Dims", "dims_of", "Plan",
            "reshape_and_cache", "attention_varlen", "validate_inputs", "status_string", "Trace",
            "workspace_for",
            "PA_OK", "PA_ERR_NULL", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "PA_ERR_ALIGN",
-           "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_BOUNDS", "PA_ERR_CUDA", "PA_ERR_PLAN"]
+           "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_BOUNDS", "PA_ERR_CUDA", "PA_ERR_PLAN",
+           "PA_ERR_TOO_LARGE", "attention_varlen_noalloc", "noalloc_scratch_bytes"]
 
 PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE, PA_ERR_ALIGN = 0, -1, -2, -3, -4
 PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_BOUNDS, PA_ERR_CUDA, PA_ERR_PLAN = -5, -6, -7, -8, -9
+PA_ERR_TOO_LARGE = -10
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libpa.so")
@@ -88,6 +90,8 @@ def load_library():
             "pa_plan_destroy": (None, [P]),
             "pa_attention_varlen": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P]),
             "pa_attention_varlen_ex": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P, P]),
+            "pa_attention_varlen_noalloc": (I, [P, P, P, P, P, P, F, P, DP, P, P]),
+            "pa_noalloc_scratch_bytes": (SZ, []),
             "pa_validate_scratch_bytes": (SZ, [DP]),
             "pa_validate_inputs": (I, [P, P, P, P, DP, P, SZ, P]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -283,6 +287,30 @@ def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, 
     else:
         trace.arm(stream if stream is not None else torch.cuda.current_stream())
         _check(lib.pa_attention_varlen_ex(*args, ctypes.byref(trace)), "pa_attention_varlen_ex")
+    return out
+
+
+def noalloc_scratch_bytes() -> int:
+    """Size of the fixed device array pa_attention_varlen_noalloc uses."""
+    return int(load_library().pa_noalloc_scratch_bytes())
+
+
+def attention_varlen_noalloc(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale,
+                             out, plan: Plan, stream=None) -> torch.Tensor:
+    """pa_attention_varlen_noalloc: the same attention with no caller workspace
+    (the library's fixed device array serves as scratch; see include/pa.h for
+    who needs this and the rules for concurrent calls)."""
+    lib = load_library()
+    d = plan.dims
+    bf = torch.bfloat16
+    if tuple(q.shape) != (d.num_tokens, d.num_q_heads, d.head_dim) or out.shape != q.shape:
+        raise PaError(PA_ERR_SHAPE, "q/out shape does not match the plan")
+    _check(lib.pa_attention_varlen_noalloc(
+        _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf), _dev_ptr(v_cache, "v_cache", bf),
+        _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(cu_seqlens_q, "cu_seqlens_q", torch.int32), _dev_ptr(seq_lens, "seq_lens", torch.int32),
+        ctypes.c_float(scale), _dev_ptr(out, "out", bf), ctypes.byref(d), plan.handle,
+        _stream_ptr(stream)), "pa_attention_varlen_noalloc")
     return out
 
 

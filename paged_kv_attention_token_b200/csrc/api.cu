@@ -68,6 +68,9 @@ extern "C" const char *pa_status_string(int status) {
         case PA_ERR_BOUNDS: return "input precondition violated (slot, block id or segment bounds)";
         case PA_ERR_CUDA: return "CUDA error";
         case PA_ERR_PLAN: return "plan does not match the call";
+        case PA_ERR_TOO_LARGE:
+            return "call needs more scratch than the 16 MiB no-alloc array holds; "
+                   "use pa_attention_varlen with a workspace";
         default: return "unknown status";
     }
 }
