@@ -104,8 +104,8 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  * device arrays will hold) it splits the step into balanced GPU work:
  * segments with q_len <= 16 (decodes, speculative-verification shapes) are
  * cut into equal runs of 16-token KV blocks over all query rows and kv heads
- * (split-KV), each run one warp's work, with a combine step for rows cut in
- * several runs; longer segments are cut into 128-query tiles per query head
+ * (split-KV), one run per CTA and SM, the partials of rows cut between runs
+ * being merged by the last CTA to finish them; longer segments are cut into 128-query tiles per query head
  * for the tensor-core prefill kernel, longest tiles first.
  *   h_cu_seqlens_q  host [S+1] int32
  *   h_seq_lens      host [S] int32
@@ -209,6 +209,15 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
                            const int32_t *d_seq_lens, float scale, void *d_out,
                            const pa_dims *dims, const pa_plan *plan, void *d_workspace,
                            size_t workspace_bytes, void *stream, const pa_trace *trace);
+
+/*
+ * Status word of a workspace after a pa_attention_varlen call: waits for
+ * `stream`, then copies the word to *status.  0 means no error; bit 0 means
+ * some wait inside a kernel gave up after about a second (the kernels never
+ * block longer, and the affected outputs are undefined).  The word is reset
+ * by every call that uses the workspace.
+ */
+int pa_workspace_status(const void *d_workspace, void *stream, uint32_t *status);
 
 /*
  * Opt-in check of the data-dependent preconditions, on the device, then a

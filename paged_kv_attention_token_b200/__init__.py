@@ -26,7 +26,7 @@ __all__ = ["load_library", "library_path", "PaError", "Dims", "dims_of", "Plan",
            "workspace_for",
            "PA_OK", "PA_ERR_NULL", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "PA_ERR_ALIGN",
            "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_BOUNDS", "PA_ERR_CUDA", "PA_ERR_PLAN",
-           "PA_ERR_TOO_LARGE", "attention_varlen_noalloc", "noalloc_scratch_bytes"]
+           "PA_ERR_TOO_LARGE", "attention_varlen_noalloc", "noalloc_scratch_bytes", "workspace_status"]
 
 PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE, PA_ERR_ALIGN = 0, -1, -2, -3, -4
 PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_BOUNDS, PA_ERR_CUDA, PA_ERR_PLAN = -5, -6, -7, -8, -9
@@ -92,6 +92,7 @@ def load_library():
             "pa_attention_varlen_ex": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P, P]),
             "pa_attention_varlen_noalloc": (I, [P, P, P, P, P, P, F, P, DP, P, P]),
             "pa_noalloc_scratch_bytes": (SZ, []),
+            "pa_workspace_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "pa_validate_scratch_bytes": (SZ, [DP]),
             "pa_validate_inputs": (I, [P, P, P, P, DP, P, SZ, P]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -288,6 +289,15 @@ def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, 
         trace.arm(stream if stream is not None else torch.cuda.current_stream())
         _check(lib.pa_attention_varlen_ex(*args, ctypes.byref(trace)), "pa_attention_varlen_ex")
     return out
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Error bits the last attention call left in a workspace (0 = none);
+    waits for the stream."""
+    st = ctypes.c_uint32(0)
+    _check(load_library().pa_workspace_status(_dev_ptr(workspace, "workspace"), _stream_ptr(stream),
+                                              ctypes.byref(st)), "pa_workspace_status")
+    return int(st.value)
 
 
 def noalloc_scratch_bytes() -> int:

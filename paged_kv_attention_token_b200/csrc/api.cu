@@ -165,6 +165,8 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.partial_ml = reinterpret_cast<float2 *>(ws + w.partial_ml);
         p.units = reinterpret_cast<const DecodeUnit *>(ws + w.units);
         p.rows = reinterpret_cast<const DecodeRow *>(ws + w.rows);
+        p.combine = reinterpret_cast<CombineRow *>(ws + w.combine);
+        p.status = reinterpret_cast<uint32_t *>(ws + w.header);
         p.num_units = plan->num_units;
         p.num_q_heads = d.num_q_heads;
         p.num_kv_heads = d.num_kv_heads;
@@ -173,15 +175,20 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.scale_log2 = scale_log2;
         if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 2, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (launch_combine(reinterpret_cast<const CombineRow *>(ws + w.combine), p.rows,
-                           p.partial_o, p.partial_ml, p.out, plan->num_combine, plan->group,
-                           d.num_q_heads, d.num_kv_heads, d.head_dim, stream) != cudaSuccess)
-            return PA_ERR_CUDA;
     } else if (mark(trace, 2, stream) != cudaSuccess) {
         return PA_ERR_CUDA;
     }
     if (mark(trace, 3, stream) != cudaSuccess || mark(trace, 4, stream) != cudaSuccess ||
         mark(trace, 5, stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+extern "C" int pa_workspace_status(const void *workspace, void *stream_, uint32_t *status) {
+    if (!workspace || !status) return PA_ERR_NULL;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
         return PA_ERR_CUDA;
     return PA_OK;
 }

@@ -1,5 +1,6 @@
 // Kernel launchers of libpa.so (internal).
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -18,6 +19,8 @@ struct DecodeParams {
     float2 *partial_ml;     // [pieces][G]: (max in log2 units, sum)
     const DecodeUnit *units;
     const DecodeRow *rows;
+    CombineRow *combine;        // tickets live here; zero at upload
+    uint32_t *status;           // workspace status word (error bits), zero at upload
     int num_units;
     int num_q_heads;
     int num_kv_heads;
@@ -32,11 +35,6 @@ cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t
                                      cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);
-
-cudaError_t launch_combine(const CombineRow *combine, const DecodeRow *rows, const float *partial_o,
-                           const float2 *partial_ml, __nv_bfloat16 *out, int num_combine,
-                           int group, int num_q_heads, int num_kv_heads, int head_dim,
-                           cudaStream_t stream);
 
 // Data-dependent precondition checks; writes a nonzero flag word on failure.
 cudaError_t launch_validate(const int64_t *slots, const int32_t *block_tables,

@@ -9,7 +9,7 @@
 // (split-KV in the flash-decoding manner, balanced like stream-K), so every
 // warp moves the same number of KV bytes whatever the length mix.  A row cut
 // across several runs leaves one partial (unnormalised O, running max and
-// sum) per run; the combine step merges them.
+// sum) per run; the last run to finish merges them (see CombineRow).
 //
 // Prefill side (longer segments): 128-query tiles per query head, ordered by
 // the number of 128-key tiles they read, longest first.
@@ -28,8 +28,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Fewest KV blocks one decode warp is given, so that per-warp fixed costs
-// (loading q, the final write) stay small against the streaming.
+// Fewest KV blocks one decode warp is given, so that its fixed costs (loading
+// q, the final write or merge) stay small against the streaming.
 constexpr int64_t kMinBlocksPerUnit = 4;
 
 // Waits until the last table copy queued from this plan has executed.
@@ -102,10 +102,6 @@ int check_dims(const pa_dims *d) {
 
 }  // namespace
 
-namespace pa {
-int decode_warps_per_sm(int head_dim) { return head_dim <= 64 ? 16 : 8; }
-}  // namespace pa
-
 extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa_dims *dims,
                              int device, pa_plan **out) {
     if (!out) return PA_ERR_NULL;
@@ -148,7 +144,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
         if (L <= pa::kDecodeMaxQLen || !pa::prefill_kernel_available()) {
             for (int j = 0; j < L; ++j)
                 for (int g = 0; g < Hkv; ++g)
-                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow});
+                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, {0, 0, 0}});
         } else {
             for (int q0 = 0; q0 < L; q0 += pa::kPrefillTileM) {
                 const int last = std::min(L, q0 + pa::kPrefillTileM) - 1;
@@ -170,7 +166,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     const int64_t total = prefix[R];
     int64_t P = 0;
     if (total > 0) {
-        const int64_t max_units = (int64_t)p->num_sms * pa::decode_warps_per_sm(d.head_dim);
+        const int64_t max_units = (int64_t)p->num_sms * pa::decode_units_per_sm(d.head_dim);
         P = std::max<int64_t>(1, std::min(max_units, cdiv(total, kMinBlocksPerUnit)));
     }
     std::vector<pa::DecodeUnit> units(P + 1);
@@ -197,6 +193,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
             const int32_t count = (int32_t)(v - u + 1);
             if (count > 1) {
                 rows[r].slot_base = piece_base - (int32_t)u;
+                rows[r].combine = (int32_t)combine.size();
                 combine.push_back({(int32_t)r, piece_base, count, 0});
                 piece_base += count;
             }
@@ -212,6 +209,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
 
     pa::WorkspaceLayout &w = p->ws;
     size_t off = 0;
+    w.header = off;  off = pa::kHeaderBytes;
     w.units = off;   off = align_up(off + sizeof(pa::DecodeUnit) * units.size(), pa::kWorkspaceAlign);
     w.rows = off;    off = align_up(off + sizeof(pa::DecodeRow) * rows.size(), pa::kWorkspaceAlign);
     w.combine = off; off = align_up(off + sizeof(pa::CombineRow) * combine.size(), pa::kWorkspaceAlign);

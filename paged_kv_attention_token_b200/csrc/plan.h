@@ -31,6 +31,8 @@ struct DecodeRow {
     int32_t n_keys;     // keys this query sees: p + 1
     int32_t slot_base;  // kUnsplitRow: one warp covers the row and writes out
                         // directly; else partial slot of unit u is slot_base + u
+    int32_t combine;    // index of the row's CombineRow (split rows only)
+    int32_t pad[3];
 };
 
 // A decode warp's work: flat (row, block) range [start, next unit's start).
@@ -39,12 +41,14 @@ struct DecodeUnit {
     int32_t block;
 };
 
-// A row cut across several units: the combine step merges its partials.
+// A row cut across several units.  Each unit writes its partial, then takes
+// a ticket from `arrived` (zero in the uploaded tables); the unit that takes
+// the last ticket merges the partials and writes the row.  Nobody waits.
 struct CombineRow {
     int32_t row;
     int32_t piece_base;
     int32_t piece_count;
-    int32_t pad;
+    int32_t arrived;
 };
 
 // One prefill tile: up to 128 consecutive queries of one segment, one query
@@ -57,7 +61,8 @@ struct PrefillTile {
 };
 
 struct WorkspaceLayout {
-    size_t units = 0, rows = 0, combine = 0, tiles = 0;  // byte offsets
+    // byte offsets; the header (status word first) is at offset 0
+    size_t header = 0, units = 0, rows = 0, combine = 0, tiles = 0;
     size_t table_bytes = 0;                              // bytes copied from the plan
     size_t partial_o = 0, partial_ml = 0;                // scratch offsets
     size_t total = 0;
@@ -79,7 +84,7 @@ struct pa_plan {
     int32_t num_tiles = 0;
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::WorkspaceLayout ws;
-    // Image of [units | rows | combine | tiles], copied into the workspace by
+    // Image of [header | units | rows | combine | tiles], copied into the workspace by
     // every attention call.  Page-locked when a device is present, so that the
     // copy is truly asynchronous; the event is recorded after each copy, and a
     // rebuild or destroy waits on it before touching the buffer.
@@ -91,8 +96,9 @@ struct pa_plan {
 };
 
 namespace pa {
-// Decode warps a launch can keep resident per SM for a head dim.
-int decode_warps_per_sm(int head_dim);
+constexpr size_t kHeaderBytes = 256;  // status word and reserved space
+// Decode warps resident per SM for a head dim (one planner unit per warp).
+int decode_units_per_sm(int head_dim);
 // SM count of a device (cached per process; 148 when it cannot be read).
 int device_sm_count(int device);
 // Whether long segments go to the tensor-core prefill kernel.

@@ -34,6 +34,7 @@ def run_step(batch):
     out = torch.full_like(batch.q, float("nan"))
     pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws)
     torch.cuda.synchronize()
+    assert pa.workspace_status(ws) == 0          # no bounded wait gave up
     return kc, vc, out, plan
 
 
