@@ -48,8 +48,6 @@ int device_sm_count(int device) {
     return n;
 }
 
-bool prefill_kernel_available() { return false; }
-
 }  // namespace pa
 
 using namespace pa;
@@ -178,9 +176,27 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
     } else if (mark(trace, 2, stream) != cudaSuccess) {
         return PA_ERR_CUDA;
     }
-    if (mark(trace, 3, stream) != cudaSuccess || mark(trace, 4, stream) != cudaSuccess ||
-        mark(trace, 5, stream) != cudaSuccess)
-        return PA_ERR_CUDA;
+    if (mark(trace, 3, stream) != cudaSuccess || mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (plan->num_tiles > 0) {
+        PrefillParams pp;
+        pp.q = static_cast<const __nv_bfloat16 *>(q);
+        pp.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+        pp.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+        pp.block_tables = block_tables;
+        pp.cu_seqlens_q = cu_seqlens_q;
+        pp.seq_lens = seq_lens;
+        pp.out = static_cast<__nv_bfloat16 *>(out);
+        pp.tiles = reinterpret_cast<const PrefillTile *>(ws + w.tiles);
+        pp.status = reinterpret_cast<uint32_t *>(ws + w.header);
+        pp.num_tiles = plan->num_tiles;
+        pp.num_q_heads = d.num_q_heads;
+        pp.num_kv_heads = d.num_kv_heads;
+        pp.group = plan->group;
+        pp.max_blocks_per_seq = d.max_blocks_per_seq;
+        pp.scale_log2 = scale_log2;
+        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+    }
+    if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;
     return PA_OK;
 }
 

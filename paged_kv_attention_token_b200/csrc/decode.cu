@@ -165,9 +165,11 @@ __device__ __forceinline__ void attend_step(RowState<D, NT> &st, uint32_t stage,
             for (int nb = 0; nb < NB; ++nb) {
                 const float p0 = fast_exp2(s[nb][nt][e] - st.m[nt][e]);
                 const float p1 = fast_exp2(s[nb][nt][e + 2] - st.m[nt][e]);
-                s[nb][nt][e] = p0;
-                s[nb][nt][e + 2] = p1;
-                lsum += p0 + p1;
+                // the PV product uses these rounded to bf16: sum the same values
+                const uint32_t pr = pack_bf16x2(p0, p1);
+                s[nb][nt][e] = __uint_as_float(pr << 16);
+                s[nb][nt][e + 2] = __uint_as_float(pr & 0xffff0000u);
+                lsum += bf16x2_sum(pr);
             }
             st.l[nt][e] = st.l[nt][e] * alpha[nt][e] + lsum;
         }

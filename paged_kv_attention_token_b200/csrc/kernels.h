@@ -36,6 +36,26 @@ cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);
 
+struct PrefillParams {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_cache;
+    const __nv_bfloat16 *v_cache;
+    const int32_t *block_tables;
+    const int32_t *cu_seqlens_q;
+    const int32_t *seq_lens;
+    __nv_bfloat16 *out;
+    const PrefillTile *tiles;
+    uint32_t *status;
+    int num_tiles;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;
+    int max_blocks_per_seq;
+    float scale_log2;
+};
+
+cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream);
+
 // Data-dependent precondition checks; writes a nonzero flag word on failure.
 cudaError_t launch_validate(const int64_t *slots, const int32_t *block_tables,
                             const int32_t *cu_seqlens_q, const int32_t *seq_lens,

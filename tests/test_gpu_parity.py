@@ -144,6 +144,32 @@ def test_custom_shapes_all_rows(cuda_lib, case, q_gain):
     assert_parity(gpu_rows(out, tok), want, f"case {case} q_gain={q_gain} plan={plan.info()}")
 
 
+PREFILL = [
+    # (q_lens, seq_lens, Hq, Hkv, D): segments with q_len > 16 run on the
+    # tensor-core prefill kernel
+    ([300], [300], 8, 2, 128),                          # fresh prompt, 3 query tiles, ragged tail
+    ([200], [1000], 12, 2, 128),                        # chunk on 800 cached tokens (offset not /128)
+    ([129, 17], [129, 517], 4, 4, 64),                  # D = 64, tile edge + chunk of 17
+    ([1000], [1000], 16, 1, 64),                        # G = 16
+    ([1, 1, 130, 1, 64], [700, 33, 3000, 5, 64], 12, 2, 128),  # mixed with decodes
+    ([17], [17], 6, 6, 128),                            # smallest prefill, G = 1
+    ([256], [4096], 12, 2, 128),                        # long prior context, 32 key tiles
+]
+
+
+@pytest.mark.parametrize("case", range(len(PREFILL)))
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_prefill_tensor_core_all_rows(cuda_lib, case, q_gain):
+    q_lens, seq_lens, Hq, Hkv, D = PREFILL[case]
+    nb = sum(-(-s // 16) for s in seq_lens) + 64
+    lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, nb, seed=200 + case)
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, plan = run_step(b)
+    assert plan.info()["num_prefill_tiles"] > 0
+    tok, want = oracle_subset(b, range(lay.num_seqs))
+    assert_parity(gpu_rows(out, tok), want, f"prefill case {case} q_gain={q_gain} plan={plan.info()}")
+
+
 def test_split_rows_are_exercised(cuda_lib):
     q_lens, seq_lens, Hq, Hkv, D = CUSTOM[1]
     lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, 600, seed=101)
