@@ -105,8 +105,9 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  * segments with q_len <= 16 (decodes, speculative-verification shapes) are
  * cut into equal runs of 16-token KV blocks over all query rows and kv heads
  * (split-KV), one run per CTA and SM, the partials of rows cut between runs
- * being merged by the last CTA to finish them; longer segments are cut into 128-query tiles per query head
- * for the tensor-core prefill kernel, longest tiles first.
+ * being merged by the last CTA to finish them; longer segments are cut into
+ * 128-query tiles for pairs of query heads sharing a kv head, for the
+ * tensor-core prefill kernel, longest tiles first.
  *   h_cu_seqlens_q  host [S+1] int32
  *   h_seq_lens      host [S] int32
  *   dims            host; T, S, Hq, Hkv, D, B are used
@@ -139,7 +140,7 @@ typedef struct {
     int32_t num_decode_units;     /* warps of the split-KV kernel */
     int32_t num_partials;         /* partial results the combine step merges */
     int32_t num_combine_rows;     /* rows cut across more than one warp */
-    int32_t num_prefill_tiles;    /* (128-query tile, query head) items */
+    int32_t num_prefill_tiles;    /* (128-query tile, query-head pair) items */
     int64_t decode_kv_blocks;     /* sum over decode rows of ceil(keys / 16) */
     int64_t prefill_causal_pairs; /* (query, visible key) pairs per query head */
     uint64_t table_bytes;         /* plan tables copied into the workspace per call */

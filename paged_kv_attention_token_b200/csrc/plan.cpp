@@ -11,8 +11,9 @@
 // across several runs leaves one partial (unnormalised O, running max and
 // sum) per run; the last run to finish merges them (see CombineRow).
 //
-// Prefill side (longer segments): 128-query tiles per query head, ordered by
-// the number of 128-key tiles they read, longest first.
+// Prefill side (longer segments): 128-query tiles for pairs of query heads
+// that share a kv head, ordered by the number of 128-key tiles they read,
+// longest first.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
@@ -149,7 +150,10 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
             for (int q0 = 0; q0 < L; q0 += pa::kPrefillTileM) {
                 const int last = std::min(L, q0 + pa::kPrefillTileM) - 1;
                 const int kv_tiles = (int)cdiv(n - L + last + 1, pa::kPrefillTileN);
-                for (int h = 0; h < d.num_q_heads; ++h) tiles.push_back({i, q0, h, kv_tiles});
+                const int G = d.num_q_heads / d.num_kv_heads;
+                for (int g = 0; g < Hkv; ++g)
+                    for (int h = g * G; h < (g + 1) * G; h += 2)
+                        tiles.push_back({i, q0, h, kv_tiles, std::min(2, (g + 1) * G - h), {0, 0, 0}});
             }
             for (int j = 0; j < L; ++j) p->prefill_pairs += n - L + j + 1;
         }

@@ -51,13 +51,15 @@ struct CombineRow {
     int32_t arrived;
 };
 
-// One prefill tile: up to 128 consecutive queries of one segment, one query
-// head.
+// One prefill work item: up to 128 consecutive queries of one segment for one
+// or two query heads that share a kv head.
 struct PrefillTile {
     int32_t seq;        // segment index
     int32_t q_start;    // first query of the tile within the segment (j)
-    int32_t head;       // query head
+    int32_t head;       // first query head
     int32_t n_kv_tiles; // 128-key tiles the tile reads (work estimate)
+    int32_t num_heads;  // 1 or 2 (head and head + 1)
+    int32_t pad[3];
 };
 
 struct WorkspaceLayout {
