@@ -72,6 +72,27 @@ def step_bytes(lay: W.Layout) -> dict:
     return {"kv": kv, "qo": qo, "scatter": scatter, "meta": meta, "total": kv + qo + scatter + meta}
 
 
+def decode_prefill_split(lay: W.Layout):
+    """Algorithmic work of the two kernels: the decode kernel's distinct KV
+    bytes (+ q/out of its rows) and the prefill kernel's flops (4 D per
+    causal (query, key) pair and query head) and bytes."""
+    Hq, Hkv, D = lay.num_q_heads, lay.num_kv_heads, lay.head_dim
+    per_tok = 2 * Hkv * D * 2
+    dec = lay.q_lens <= 16
+    dec_tokens = int(lay.q_lens[dec].sum())
+    if lay.shared_prefix_blocks and dec.all():
+        kv_dec = lay.kv_bytes_read()
+    else:
+        kv_dec = per_tok * int(lay.seq_lens[dec].astype(np.int64).sum())
+    pairs = 0
+    for L, n in zip(lay.q_lens[~dec].astype(np.int64), lay.seq_lens[~dec].astype(np.int64)):
+        pairs += int(L * (n - L) + L * (L + 1) // 2)
+    flops = 4 * D * Hq * pairs
+    kv_pre = per_tok * int(lay.seq_lens[~dec].astype(np.int64).sum())
+    return {"decode_bytes": kv_dec + 2 * dec_tokens * Hq * D * 2, "prefill_flops": flops,
+            "prefill_bytes": kv_pre + 2 * int(lay.q_lens[~dec].sum()) * Hq * D * 2}
+
+
 def is_decode_workload(lay: W.Layout) -> bool:
     return bool(np.all(lay.q_lens <= 1))
 
@@ -313,8 +334,8 @@ def run_ours(args):
     ws = pa.workspace_for(plan0, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + \
-        (1 if info["num_combine_rows"] else 0) + (1 if info["num_prefill_tiles"] else 0)
+    # scatter, split-KV decode (split rows are merged inside it), prefill
+    launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + (1 if info["num_prefill_tiles"] else 0)
 
     # two plans rebuilt in turn, as an engine keeps them across steps
     plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local), pa.Plan(h_cu, h_sl, dims, device=local)]
@@ -390,14 +411,35 @@ def run_ours(args):
     comb_ms = statistics.mean(s["combine"] for s in other)
     copy_ms = statistics.mean(s["table_copy"] for s in other)
     prefill_ms = statistics.mean(s["prefill"] for s in other)
-    dec_bytes = acct["kv"] + acct["qo"] + acct["meta"]
-    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    src_hash = kernel_source_hash(["decode.cu", "common.cuh", "kernels.h", "plan.h"])
-    roofline = {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved,
-                "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "traffic": profiled_traffic("decode_kernel", args.workload, src_hash),
-                "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash}
+    split = decode_prefill_split(lay)
+    roofline_decode = roofline_prefill = None
+    dec_bytes = split["decode_bytes"]
+    if dec_bytes and dec_ms > 0:
+        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+        src_hash = kernel_source_hash(["decode.cu", "common.cuh", "kernels.h", "plan.h"])
+        roofline_decode = {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved,
+                           "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
+                           "frac": achieved / peaks["hbm_gbs"],
+                           "traffic": profiled_traffic("decode_kernel", args.workload, src_hash),
+                           "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash}
+    if split["prefill_flops"] and prefill_ms > 0:
+        tflops = split["prefill_flops"] / (prefill_ms * 1e-3) / 1e12
+        pre_hash = kernel_source_hash(["prefill.cu", "common.cuh", "kernels.h", "plan.h"])
+        roofline_prefill = {"bound": "tensor", "kernel": "prefill_kernel", "achieved": tflops,
+                            "peak": peaks["bf16_tflops"], "peak_kind": peak_kind + " (burst bf16)",
+                            "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                            "traffic": profiled_traffic("prefill_kernel", args.workload, pre_hash),
+                            "algorithmic_flops": split["prefill_flops"], "ms": prefill_ms,
+                            "source_hash": pre_hash}
+    # "roofline" is the dominant kernel's: the one with the longer device time
+    cands = [r for r in (roofline_decode, roofline_prefill) if r is not None]
+    roofline = max(cands, key=lambda r: r["ms"]) if cands else None
+    # whole step against its roofline: the slower of the tensor-bound prefill
+    # time and the HBM-bound time of every algorithmic byte of the step
+    t_roof = max(split["prefill_flops"] / (peaks["bf16_tflops"] * 1e12),
+                 acct["total"] / (peaks["hbm_gbs"] * 1e9))
+    step_roofline = {"t_roofline_ms": t_roof * 1e3, "t_measured_ms": ms_per_step,
+                     "frac": t_roof * 1e3 / ms_per_step}
 
     # e2e: public API with host buffers; H2D of the step's inputs, D2H of out
     e2e = None
@@ -451,6 +493,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "shape": lay.description,
                        "bytes_per_step": acct["total"], "kv_bytes_per_step": acct["kv"],
+                       "kv_bytes_logical_per_step": lay.kv_bytes_logical(),
                        "tokens_per_step": lay.num_tokens,
                        "l2": "flushed before every timed step (1 GiB write, outside the events)",
                        "plan_us_host": 1e6 * statistics.median(plan_times),
@@ -460,6 +503,9 @@ def run_ours(args):
                        "parallelism": f"replicas x{world} (weak: one batch per GPU)",
                        "wall_s_timed_region": wall},
             "roofline": roofline,
+            "roofline_decode": roofline_decode,
+            "roofline_prefill": roofline_prefill,
+            "step_roofline": step_roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,

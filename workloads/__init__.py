@@ -198,6 +198,13 @@ def _prefix_llama3_70b(seed):
                          "prefix_llama3_70b_b128", shared_prefix_blocks=256)
 
 
+def _prefill_qwen25(seed):
+    # the mixed step's prefill side alone, at a size a profiler captures in
+    # seconds: four fresh 2048-token prompts with the Qwen2.5-1.5B head shape
+    return custom_layout(np.full(4, 2048, np.int32), np.full(4, 2048, np.int32), 12, 2, 128,
+                         4 * 128 + 16, seed + 1, "prefill_qwen25_1p5b_4x2048")
+
+
 WORKLOADS = {
     "tiny_mixed": (_tiny_mixed, 1001,
                    "3 requests, seq 17/40/6, q 1/1/6; Hq 4, Hkv 2, D 64; pool 64 blocks"),
@@ -211,6 +218,8 @@ WORKLOADS = {
     "prefix_llama3_70b_b128": (_prefix_llama3_70b, 1005,
                                "128 decodes sharing a 4096-token prefix (256 blocks) + suffix "
                                "U[256,1024]; Hq 64, Hkv 8, D 128; pool 16384 blocks"),
+    "prefill_qwen25_1p5b_4x2048": (_prefill_qwen25, 1006,
+                                   "4 fresh 2048-token prompts; Hq 12, Hkv 2, D 128; pool 528 blocks"),
 }
 
 
