@@ -145,6 +145,9 @@ typedef struct {
     int64_t prefill_causal_pairs; /* (query, visible key) pairs per query head */
     uint64_t table_bytes;         /* plan tables copied into the workspace per call */
     uint64_t workspace_bytes;     /* = pa_plan_workspace_bytes */
+    int32_t num_staged_kv_tiles;  /* 128-key K/V tiles of prefill segments gathered
+                                     into the workspace (per kv head) */
+    int32_t num_prefill_ctas;     /* persistent CTAs of the prefill kernel */
 } pa_plan_info;
 int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
 

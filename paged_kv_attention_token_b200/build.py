@@ -12,6 +12,7 @@ import argparse
 import concurrent.futures as cf
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -45,6 +46,30 @@ def _stale(obj: str, src: str, newest_header: float) -> bool:
     return t < os.path.getmtime(src) or t < newest_header
 
 
+# Kernels that move registers between warpgroups with setmaxnreg: a split
+# whose sum exceeds what the CTA was launched with would wait forever, so the
+# register count ptxas gives the kernel is checked against the split the
+# source assumes before the library is linked.
+REG_SPLIT_SOURCES = {"prefill.cu": "prefill_kernel"}
+
+
+def check_register_split(src: str, ptxas_log: str) -> None:
+    text = open(src).read()
+    want = {k: int(re.search(rf"{k} = (\d+);", text).group(1)) for k in ("kLaunchRegs", "kRegsLow", "kRegsHigh")}
+    threads = int(re.search(r"kThreads = (\d+);", text).group(1))
+    kernel = REG_SPLIT_SOURCES[os.path.basename(src)]
+    found = re.findall(rf"Compiling entry function '([^']*{kernel}[^']*)'.*?Used (\d+) registers", ptxas_log, re.S)
+    if not found:
+        raise RuntimeError(f"{os.path.basename(src)}: no ptxas register report for {kernel}")
+    for name, regs in found:
+        regs = int(regs)
+        low_threads = 128
+        need = low_threads * want["kRegsLow"] + (threads - low_threads) * want["kRegsHigh"]
+        if regs != want["kLaunchRegs"] or need > threads * regs:
+            raise RuntimeError(f"{name}: ptxas gives {regs} registers per thread at launch; the source assumes "
+                               f"{want['kLaunchRegs']} and a split needing {need} of {threads * regs}")
+
+
 def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) -> str:
     os.makedirs(BUILD, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
@@ -57,7 +82,7 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) 
         objs.append(obj)
         if force or _stale(obj, src, hdr):
             cmd = [cc, *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
-            if verbose_ptxas and src.endswith(".cu"):
+            if (verbose_ptxas and src.endswith(".cu")) or os.path.basename(src) in REG_SPLIT_SOURCES:
                 cmd.insert(1, "-Xptxas=-v")
             jobs.append((src, cmd))
 
@@ -69,6 +94,14 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) 
     failed = False
     with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
         for src, cmd, r in ex.map(run, jobs):
+            if r.returncode == 0 and os.path.basename(src) in REG_SPLIT_SOURCES:
+                try:
+                    check_register_split(src, r.stderr)
+                except RuntimeError as e:
+                    os.remove(os.path.join(BUILD, os.path.basename(src) + ".o"))
+                    failed = True
+                    sys.stderr.write(f"[build] FAILED register check: {e}\n")
+                    continue
             if r.returncode != 0:
                 failed = True
                 sys.stderr.write(f"[build] FAILED {os.path.basename(src)}\n{' '.join(cmd)}\n{r.stdout}{r.stderr}\n")

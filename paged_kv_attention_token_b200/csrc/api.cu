@@ -187,8 +187,15 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         pp.seq_lens = seq_lens;
         pp.out = static_cast<__nv_bfloat16 *>(out);
         pp.tiles = reinterpret_cast<const PrefillTile *>(ws + w.tiles);
+        pp.cta_start = reinterpret_cast<const int32_t *>(ws + w.cta_start);
+        pp.num_ctas = plan->num_prefill_ctas;
+        pp.stages = reinterpret_cast<const StageTile *>(ws + w.stages);
+        pp.staged = ws + w.staged;
+        pp.num_stages = plan->num_stages;
         pp.status = reinterpret_cast<uint32_t *>(ws + w.header);
         pp.num_tiles = plan->num_tiles;
+        pp.num_tokens = d.num_tokens;
+        pp.num_blocks = d.num_blocks;
         pp.num_q_heads = d.num_q_heads;
         pp.num_kv_heads = d.num_kv_heads;
         pp.group = plan->group;

@@ -44,9 +44,16 @@ struct PrefillParams {
     const int32_t *cu_seqlens_q;
     const int32_t *seq_lens;
     __nv_bfloat16 *out;
-    const PrefillTile *tiles;
+    const PrefillTile *tiles;  // grouped by CTA
+    const int32_t *cta_start;  // CTA c owns tiles [cta_start[c], cta_start[c + 1])
+    const StageTile *stages;   // the gather kernel's list
+    uint8_t *staged;          // staged K/V tiles (workspace)
     uint32_t *status;
     int num_tiles;
+    int num_ctas;
+    int num_stages;
+    int num_tokens;  // rows of q (extent of its TMA descriptor)
+    int num_blocks;  // blocks of the pool (extent of the cache descriptors)
     int num_q_heads;
     int num_kv_heads;
     int group;

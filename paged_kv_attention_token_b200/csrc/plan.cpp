@@ -12,10 +12,17 @@
 // sum) per run; the last run to finish merges them (see CombineRow).
 //
 // Prefill side (longer segments): 128-query tiles for pairs of query heads
-// that share a kv head, ordered by the number of 128-key tiles they read,
-// longest first.
+// that share a kv head, dealt to at most one persistent CTA per SM by
+// greedy longest-processing-time assignment (each tile, longest first, goes
+// to the CTA with the least work so far; a tile costs its 128-key tiles plus
+// a fixed start/finish overhead); and, per segment and kv head, the list of
+// 128-key tiles of K/V that a gather kernel stages from the paged cache into
+// the workspace for them.
 #include <algorithm>
 #include <cstdlib>
+#include <functional>
+#include <queue>
+#include <utility>
 #include <cstring>
 #include <new>
 
@@ -28,6 +35,10 @@ namespace {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Start/finish cost of a prefill tile in units of 128-key steps (Q load,
+// first S, output write-back), for the CTA assignment.
+constexpr int64_t kTileOverheadSteps = 2;
 
 // Fewest KV blocks one decode warp is given, so that its fixed costs (loading
 // q, the final write or merge) stay small against the streaming.
@@ -138,6 +149,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
 
     std::vector<pa::DecodeRow> rows;
     std::vector<pa::PrefillTile> tiles;
+    std::vector<pa::StageTile> stages;
     for (int i = 0; i < d.num_seqs; ++i) {
         const int L = h_cu[i + 1] - h_cu[i];
         const int n = h_seq[i];
@@ -147,13 +159,17 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
                 for (int g = 0; g < Hkv; ++g)
                     rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, {0, 0, 0}});
         } else {
+            const int G = d.num_q_heads / d.num_kv_heads;
+            const int nt = (int)cdiv(n, pa::kPrefillTileN);  // key tiles of the segment
+            const int base = (int)stages.size();
+            for (int g = 0; g < Hkv; ++g)
+                for (int j = 0; j < nt; ++j) stages.push_back({i, g, j, 0});
             for (int q0 = 0; q0 < L; q0 += pa::kPrefillTileM) {
                 const int last = std::min(L, q0 + pa::kPrefillTileM) - 1;
                 const int kv_tiles = (int)cdiv(n - L + last + 1, pa::kPrefillTileN);
-                const int G = d.num_q_heads / d.num_kv_heads;
                 for (int g = 0; g < Hkv; ++g)
                     for (int h = g * G; h < (g + 1) * G; h += 2)
-                        tiles.push_back({i, q0, h, kv_tiles, std::min(2, (g + 1) * G - h), {0, 0, 0}});
+                        tiles.push_back({i, q0, h, kv_tiles, std::min(2, (g + 1) * G - h), base + g * nt, {0, 0}});
             }
             for (int j = 0; j < L; ++j) p->prefill_pairs += n - L + j + 1;
         }
@@ -162,6 +178,30 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
                      [](const pa::PrefillTile &a, const pa::PrefillTile &b) {
                          return a.n_kv_tiles > b.n_kv_tiles;
                      });
+    // Deal the tiles to persistent CTAs; each CTA's tiles become contiguous.
+    const int grid = (int)std::min<size_t>(tiles.size(), (size_t)p->num_sms);
+    std::vector<int32_t> cta_start(grid + 1, 0);
+    if (grid > 0) {
+        std::vector<std::vector<int32_t>> per(grid);
+        using Load = std::pair<int64_t, int>;
+        std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+        for (int c = 0; c < grid; ++c) heap.push({0, c});
+        for (size_t t = 0; t < tiles.size(); ++t) {
+            Load l = heap.top();
+            heap.pop();
+            per[l.second].push_back((int32_t)t);
+            l.first += tiles[t].n_kv_tiles + kTileOverheadSteps;
+            heap.push(l);
+        }
+        std::vector<pa::PrefillTile> dealt;
+        dealt.reserve(tiles.size());
+        for (int c = 0; c < grid; ++c) {
+            cta_start[c] = (int32_t)dealt.size();
+            for (int32_t t : per[c]) dealt.push_back(tiles[t]);
+        }
+        cta_start[grid] = (int32_t)dealt.size();
+        tiles.swap(dealt);
+    }
 
     // Cut the decode rows' blocks into equal runs.
     const int64_t R = (int64_t)rows.size();
@@ -210,6 +250,8 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     p->num_combine = (int32_t)combine.size();
     p->decode_blocks = total;
     p->num_tiles = (int32_t)tiles.size();
+    p->num_prefill_ctas = grid;
+    p->num_stages = (int32_t)stages.size();
 
     pa::WorkspaceLayout &w = p->ws;
     size_t off = 0;
@@ -218,12 +260,17 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     w.rows = off;    off = align_up(off + sizeof(pa::DecodeRow) * rows.size(), pa::kWorkspaceAlign);
     w.combine = off; off = align_up(off + sizeof(pa::CombineRow) * combine.size(), pa::kWorkspaceAlign);
     w.tiles = off;   off = align_up(off + sizeof(pa::PrefillTile) * tiles.size(), pa::kWorkspaceAlign);
+    w.cta_start = off; off = align_up(off + sizeof(int32_t) * cta_start.size(), pa::kWorkspaceAlign);
+    w.stages = off;  off = align_up(off + sizeof(pa::StageTile) * stages.size(), pa::kWorkspaceAlign);
     w.table_bytes = off;
     w.partial_o = off;
     off = align_up(off + sizeof(float) * (size_t)piece_base * p->group * d.head_dim, pa::kWorkspaceAlign);
     w.partial_ml = off;
     off = align_up(off + sizeof(float) * 2 * (size_t)piece_base * p->group, pa::kWorkspaceAlign);
-    w.total = off;
+    off = align_up(off, pa::kStagedAlign);
+    w.staged = off;
+    off += stages.size() * 2 * (size_t)pa::kPrefillTileN * d.head_dim * 2;
+    w.total = align_up(off, pa::kWorkspaceAlign);
 
     wait_upload(p);  // the previous build's tables may still be in a queued copy
     if (!reserve_tables(p, w.table_bytes)) {
@@ -238,6 +285,9 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
         std::memcpy(p->tables + w.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
     if (!tiles.empty())
         std::memcpy(p->tables + w.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
+    std::memcpy(p->tables + w.cta_start, cta_start.data(), sizeof(int32_t) * cta_start.size());
+    if (!stages.empty())
+        std::memcpy(p->tables + w.stages, stages.data(), sizeof(pa::StageTile) * stages.size());
     *out = p;
     return PA_OK;
 }
@@ -254,6 +304,8 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     info->prefill_causal_pairs = p->prefill_pairs;
     info->table_bytes = p->ws.table_bytes;
     info->workspace_bytes = p->ws.total;
+    info->num_staged_kv_tiles = p->num_stages;
+    info->num_prefill_ctas = p->num_prefill_ctas;
     return PA_OK;
 }
 

@@ -57,16 +57,32 @@ struct PrefillTile {
     int32_t seq;        // segment index
     int32_t q_start;    // first query of the tile within the segment (j)
     int32_t head;       // first query head
-    int32_t n_kv_tiles; // 128-key tiles the tile reads (work estimate)
+    int32_t n_kv_tiles; // 128-key tiles the tile reads
     int32_t num_heads;  // 1 or 2 (head and head + 1)
-    int32_t pad[3];
+    int32_t kv_base;    // staged tile index of key tile 0 of (seq, kv head)
+    int32_t pad[2];
 };
+
+// One staged key tile: keys 128 j .. 128 j + 127 of segment `seq` for one kv
+// head, K and V, gathered from the paged cache into the workspace in the
+// layout the prefill kernel's shared-memory tiles have (rows past the
+// segment's length zeroed).  Staged tile s occupies bytes
+// [2 s T, 2 s T + T) (K) and [2 s T + T, 2 (s + 1) T) (V) of the staged
+// area, T = 128 * head_dim * 2.
+struct StageTile {
+    int32_t seq;
+    int32_t kv_head;
+    int32_t tile;  // j
+    int32_t pad;
+};
+
+constexpr size_t kStagedAlign = 1024;
 
 struct WorkspaceLayout {
     // byte offsets; the header (status word first) is at offset 0
-    size_t header = 0, units = 0, rows = 0, combine = 0, tiles = 0;
+    size_t header = 0, units = 0, rows = 0, combine = 0, tiles = 0, cta_start = 0, stages = 0;
     size_t table_bytes = 0;                              // bytes copied from the plan
-    size_t partial_o = 0, partial_ml = 0;                // scratch offsets
+    size_t partial_o = 0, partial_ml = 0, staged = 0;    // scratch offsets
     size_t total = 0;
 };
 
@@ -84,9 +100,11 @@ struct pa_plan {
     int64_t decode_blocks = 0;           // sum over rows of ceil(n_keys / 16)
     // prefill part
     int32_t num_tiles = 0;
+    int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)
+    int32_t num_stages = 0;              // staged K/V key tiles
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::WorkspaceLayout ws;
-    // Image of [header | units | rows | combine | tiles], copied into the workspace by
+    // Image of [header | units | rows | combine | tiles | cta_start | stages], copied into the workspace by
     // every attention call.  Page-locked when a device is present, so that the
     // copy is truly asynchronous; the event is recorded after each copy, and a
     // rebuild or destroy waits on it before touching the buffer.

@@ -22,25 +22,40 @@
 //               tcgen05.mma operations of one thread run in issue order,
 //               which is what lets S_X(j+1) reuse the columns P_Xj was read
 //               from, and makes "S_Xj complete" imply "PV_X(j-1) complete".
-//   warps 1-3   load Q_A, Q_B once and K/V tiles (two stages) with 16-byte
-//               cp.async, 16-token blocks dealt out to the warps, through the block
-//               table, into 128-byte-swizzled tiles (rows of 64 dims x 2
-//               bytes, chunk index XORed by the row: the SWIZZLE_128B layout
-//               the MMA descriptors name; Q and K are read K-major, V
-//               MN-major).  Rows past the segment's length are written as
-//               zeros, so no NaN ever meets the tensor cores.
+//   warp 1      loads: Q of both heads once with TMA (no multicast), then
+//               K tiles into a ring of kKStages and V tiles into a ring of
+//               kVStages, K running ahead of V (K_(j+1) is issued before
+//               V_j), each tile with one bulk copy from the staged tiles.
+//               Tiles are 128-byte rows with the 128-byte swizzle the MMA
+//               descriptors name (Q and K read K-major, V MN-major).
+//
+// Staging (stage_kernel, launched first): the K/V of a prefill segment are
+// gathered once per kv head from the paged cache, through the block table,
+// into the workspace as 128-key tiles laid out exactly like the shared-memory
+// tiles, rows past the segment's length zeroed (so that P = 0 meets zeros,
+// never unused or NaN slots).  Measured on B200, TMA boxes of one 16-token
+// block fill shared memory at ~20 B per SM clock and cp.async at ~24, while
+// two 128-query heads of this kernel consume ~32 B per clock at tensor-core
+// rate; contiguous bulk copies from L2 run at ~50.  The gather moves each
+// K/V byte of a segment once more, which next to the segment's
+// (q_len x keys) work is a small fraction for any q_len above 16.
+//   warps 2-3   idle (they only give their registers to the softmax warps).
 //   warps 4-7   softmax of head A, warps 8-11 of head B: one query row per
 //               thread (warp w holds TMEM lanes 32 (w % 4) ...).  A thread
-//               reads its S row twice from TMEM (max, then exponentials),
-//               masks the causal edge by selection, works in base 2 with
+//               reads its S row once from TMEM into registers, masks the
+//               causal edge by selection, works in base 2 with
 //               scale*log2(e), moves its running max (and rescales its O row
 //               in TMEM) only when it grows by more than
 //               kPrefillRescaleThreshold, and writes P into the S columns.
-//               At the end it reads its O row, divides by its sum and writes
-//               bf16.
+//               A quarter of the exponentials are evaluated on the FMA pipe
+//               (exp2_fma), the rest on the MUFU unit, whose 16 results per
+//               SM and clock would otherwise bound the tile rate.  At the
+//               end it reads its O row, divides by its sum and writes bf16.
 // Every wait is on an mbarrier and bounded; on a timeout the kernel sets a
 // bit in the workspace status word and runs to the end without waiting,
 // after which TMEM is released.
+#include <cuda.h>
+
 #include <atomic>
 
 #include "common.cuh"
@@ -55,38 +70,46 @@ constexpr float kPrefillRescaleThreshold = 8.f;
 template <int D>
 struct PrefillCfg {
     static constexpr int kThreads = 384;
-    static constexpr int kLoadWarps = 3;  // warps 1-3
-    static constexpr int kLoaders = 32 * kLoadWarps;
-    static constexpr int kSoftA = 4;      // warps 4-7
-    static constexpr int kSoftB = 8;      // warps 8-11
+    static constexpr int kSoftB = 8;  // softmax of head A: warps 4-7, of head B: warps 8-11
+    static constexpr int kSlabs = D / 64;           // 64-dim slabs of a tile
     static constexpr int kTileBytes = 128 * D * 2;  // a Q, K or V tile
+    static constexpr int kKStages = D == 128 ? 3 : 4;
+    static constexpr int kVStages = D == 128 ? 2 : 4;
     static constexpr int kQAOff = 0;
     static constexpr int kQBOff = kTileBytes;
-    static constexpr int kKVOff = 2 * kTileBytes;  // stage s: K at kKVOff + 2 s T, V at + T
-    static constexpr int kBarOff = kKVOff + 4 * kTileBytes;
-    static constexpr int kNumBars = 13;
+    static constexpr int kKOff = 2 * kTileBytes;
+    static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+    static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+    // mbarriers
+    static constexpr int kBarQ = 0, kBarQEmpty = 1;
+    static constexpr int kBarKFull = 2;
+    static constexpr int kBarKEmpty = kBarKFull + kKStages;
+    static constexpr int kBarVFull = kBarKEmpty + kKStages;
+    static constexpr int kBarVEmpty = kBarVFull + kVStages;
+    static constexpr int kBarSA = kBarVEmpty + kVStages, kBarSB = kBarSA + 1;
+    static constexpr int kBarPA = kBarSB + 1, kBarPB = kBarPA + 1;
+    static constexpr int kBarOA = kBarPB + 1, kBarOB = kBarOA + 1;
+    static constexpr int kBarOAFree = kBarOB + 1, kBarOBFree = kBarOAFree + 1;
+    static constexpr int kNumBars = kBarOBFree + 1;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kUsed = kTmemSlotOff + 16;
-    // At least 120 KiB, so that one CTA (holding 512 TMEM columns) fits per SM.
-    static constexpr int kSmemBytes = kUsed + 1024 > 120 * 1024 ? kUsed + 1024 : 120 * 1024;
+    // + 1024 to align the base; well above half an SM's shared memory, so
+    // one CTA (holding all 512 TMEM columns) runs per SM.
+    static constexpr int kSmemBytes = kUsed + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
     static constexpr uint32_t kTmemCols = 512;
     // TMEM columns: S_A, O_A, S_B, O_B
     static constexpr uint32_t kSA = 0, kOA = 128, kSB = 256, kOB = 384;
-    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    // Register split: the kernel starts with kLaunchRegs per thread (the
+    // launch bound's cap, checked against ptxas output at build time);
+    // warpgroup 0 (MMA, TMA, idle warps) gives registers up to the two
+    // softmax warpgroups.
+    static constexpr int kLaunchRegs = 168;
+    static constexpr int kRegsLow = 104;
+    static constexpr int kRegsHigh = 200;
+    static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * kLaunchRegs, "register split");
 };
-
-__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
@@ -113,10 +136,42 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// 2^x for a pair, on the FMA pipe: x = i + f with i = round(x) and f in
+// [-1/2, 1/2]; 2^f from a cubic fitted (weighted least squares, relative
+// error) to 2^f on that interval: max relative error 7.5e-5 (~13.7 bits),
+// below the bf16 rounding P gets next.  2^i is added to the exponent field.
+// x is clamped to >= -125 so that the exponent never underflows: results
+// there are ~2^-125 instead of 0, which callers replace by 0 where a key is
+// masked.
+__device__ __forceinline__ void exp2_fma(uint64_t x2, float &e0, float &e1) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
+    float x0, x1;
+    f2_split(x2, x0, x1);
+    x2 = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t r2 = f2(kRound, kRound);
+    const uint64_t t = f2_add(x2, r2);  // kRound + round(x): round(x) in the low bits
+    const uint64_t fr = f2_sub(x2, f2_sub(t, r2));
+    uint64_t p = f2_fma(f2(0.055171508f, 0.055171508f), fr, f2(0.24261114f, 0.24261114f));
+    p = f2_fma(p, fr, f2(0.69326103f, 0.69326103f));
+    p = f2_fma(p, fr, f2(0.99992806f, 0.99992806f));
+    float p0, p1, t0, t1;
+    f2_split(p, p0, p1);
+    f2_split(t, t0, t1);
+    // shifted by 23, the low bits of t's encoding (round(x) in two's
+    // complement) become the exponent increment; the bits above fall off
+    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Row max over 32 S columns; keys > pos excluded when `masked`.
@@ -132,55 +187,66 @@ __device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], float mx, bo
 }
 
 // P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; adds the
-// rounded values to lsum (as a packed pair of partial sums).
+// rounded values to lsum (as a packed pair of partial sums).  Pairs 3, 7,
+// 11 and 15 use exp2_fma, the others ex2.approx.
 __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t &lsum,
                                           uint64_t scale2, uint64_t nm2, bool masked, int key0, int pos) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-        float x0, x1;
-        f2_split(f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2), x0, x1);
-        if (masked) {
-            if (key0 + 2 * c > pos) x0 = -INFINITY;
-            if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
+        const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
+        float e0, e1;
+        if ((c & 3) == 3) {
+            exp2_fma(x, e0, e1);
+            if (masked) {
+                if (key0 + 2 * c > pos) e0 = 0.f;
+                if (key0 + 2 * c + 1 > pos) e1 = 0.f;
+            }
+        } else {
+            float x0, x1;
+            f2_split(x, x0, x1);
+            if (masked) {
+                if (key0 + 2 * c > pos) x0 = -INFINITY;
+                if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
+            }
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
         }
-        pk[c] = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+        pk[c] = pack_bf16x2(e0, e1);
         lsum = f2_add(lsum, f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
     }
 }
 
-// Softmax of one head, one query row per thread (128 threads); the same code
-// serves both heads of the CTA.
+// Softmax of one head for one tile, one query row per thread (128 threads);
+// the same code serves both heads.  `it` counts this head's 128-key steps
+// over the CTA's tiles (the parity of s_full / p_full), `k` its tiles (the
+// parity of o_done).  After the last step the thread reads its O row from
+// TMEM, releases O (o_free) for the next tile's first PV, then divides by
+// its sum and writes bf16.
 template <int D>
-__device__ __noinline__ void softmax_head(const PrefillParams &p, uint32_t trow, uint32_t s_col, uint32_t o_col,
-                                          uint64_t *s_full, uint64_t *p_full, uint64_t *o_done, int nkv, int t,
-                                          int q_rows, int pos, int first_pos, int tok0, int head, bool &err) {
+__device__ __forceinline__ void softmax_tile(const PrefillParams &p, uint32_t trow, uint32_t s_col, uint32_t o_col,
+                                             uint64_t *s_full, uint64_t *p_full, uint64_t *o_done, uint64_t *o_free,
+                                             int nkv, uint32_t &it, uint32_t k, int t, int q_rows, int pos,
+                                             int first_pos, int tok0, int head, bool &err) {
     float m = -INFINITY, l = 0.f;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
-    for (int j = 0; j < nkv; ++j) {
-        if (!err && !mbar_wait(s_full, j & 1)) err = true;
+    for (int j = 0; j < nkv; ++j, ++it) {
+        if (!err && !mbar_wait(s_full, it & 1)) err = true;
         tc_fence_after();
         const int kbase = 128 * j;
         // only tiles that reach past the first query's position need the
         // causal mask (pos < n also covers the segment's length)
         const bool masked = kbase + 127 > first_pos;
-        // pass 1: row max of the raw scores (scale > 0 commutes with max);
-        // each TMEM load is in flight while the previous chunk is reduced
-        float mx = -INFINITY;
-        {
-            uint32_t ra[32], rb[32];
-            tmem_ld32(trow + s_col, ra);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 32, rb);
-            mx = chunk_max(ra, mx, masked, kbase, pos);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 64, ra);
-            mx = chunk_max(rb, mx, masked, kbase + 32, pos);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 96, rb);
-            mx = chunk_max(ra, mx, masked, kbase + 64, pos);
-            tmem_ld_wait();
-            mx = chunk_max(rb, mx, masked, kbase + 96, pos);
-        }
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32(trow + s_col, s0);
+        tmem_ld32(trow + s_col + 32, s1);
+        tmem_ld32(trow + s_col + 64, s2);
+        tmem_ld32(trow + s_col + 96, s3);
+        tmem_ld_wait();
+        // row max of the raw scores (scale > 0 commutes with max)
+        float mx = chunk_max(s0, -INFINITY, masked, kbase, pos);
+        mx = chunk_max(s1, mx, masked, kbase + 32, pos);
+        mx = chunk_max(s2, mx, masked, kbase + 64, pos);
+        mx = chunk_max(s3, mx, masked, kbase + 96, pos);
         mx *= p.scale_log2;
         float alpha = 1.f;
         const bool rescale = mx > m + kPrefillRescaleThreshold;
@@ -188,9 +254,27 @@ __device__ __noinline__ void softmax_head(const PrefillParams &p, uint32_t trow,
             alpha = fast_exp2(m - mx);
             m = mx;
         }
-        // O_X is stable: S_Xj completing implies PV_X(j-1) completed.  TMEM
-        // loads and stores are warp-collective, so the warp rescales if any
-        // lane needs it (alpha = 1 for the others).
+        // P = 2^(s*scale - m) as bf16, written over the S columns (P chunk
+        // i goes to columns 16 i .. 16 i + 15)
+        const uint64_t nm2 = f2(-m, -m);
+        uint64_t lsum = f2(0.f, 0.f);
+        {
+            uint32_t pk[16];
+            chunk_exp(s0, pk, lsum, scale2, nm2, masked, kbase, pos);
+            tmem_st16(trow + s_col, pk);
+            chunk_exp(s1, pk, lsum, scale2, nm2, masked, kbase + 32, pos);
+            tmem_st16(trow + s_col + 16, pk);
+            chunk_exp(s2, pk, lsum, scale2, nm2, masked, kbase + 64, pos);
+            tmem_st16(trow + s_col + 32, pk);
+            chunk_exp(s3, pk, lsum, scale2, nm2, masked, kbase + 96, pos);
+            tmem_st16(trow + s_col + 48, pk);
+        }
+        float l0, l1;
+        f2_split(lsum, l0, l1);
+        l = l * alpha + (l0 + l1);
+        // O_X is stable: S_Xj completing implies PV_X(j-1) completed; PV_Xj
+        // waits for p_full.  TMEM loads and stores are warp-collective, so
+        // the warp rescales if any lane needs it (alpha = 1 for the others).
         if (j > 0 && __any_sync(kFullMask, rescale)) {
 #pragma unroll
             for (int i = 0; i < D / 32; ++i) {
@@ -202,95 +286,107 @@ __device__ __noinline__ void softmax_head(const PrefillParams &p, uint32_t trow,
                 tmem_st32(trow + o_col + 32 * i, o);
             }
         }
-        // pass 2: P = 2^(s*scale - m) as bf16, written over the S columns
-        // already read (P chunk i goes to columns 16 i .. 16 i + 15)
-        const uint64_t nm2 = f2(-m, -m);
-        uint64_t lsum = f2(0.f, 0.f);
-        {
-            uint32_t ra[32], rb[32], pk[16];
-            tmem_ld32(trow + s_col, ra);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 32, rb);
-            chunk_exp(ra, pk, lsum, scale2, nm2, masked, kbase, pos);
-            tmem_st16(trow + s_col, pk);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 64, ra);
-            chunk_exp(rb, pk, lsum, scale2, nm2, masked, kbase + 32, pos);
-            tmem_st16(trow + s_col + 16, pk);
-            tmem_ld_wait();
-            tmem_ld32(trow + s_col + 96, rb);
-            chunk_exp(ra, pk, lsum, scale2, nm2, masked, kbase + 64, pos);
-            tmem_st16(trow + s_col + 32, pk);
-            tmem_ld_wait();
-            chunk_exp(rb, pk, lsum, scale2, nm2, masked, kbase + 96, pos);
-            tmem_st16(trow + s_col + 48, pk);
-        }
-        float l0, l1;
-        f2_split(lsum, l0, l1);
-        l = l * alpha + (l0 + l1);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
     }
-    if (!err && !mbar_wait(o_done, 0)) err = true;
+    if (!err && !mbar_wait(o_done, k & 1)) err = true;
     tc_fence_after();
-    const float inv = 1.f / l;
+    // the whole O row at once (one wait: TMEM loads queue behind the MMAs of
+    // the other head), then O is free for the next tile
+    uint32_t o[D / 32][32];
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-        uint32_t o[32];
-        tmem_ld32(trow + o_col + 32 * i, o);
-        tmem_ld_wait();
-        if (t < q_rows) {
-            __nv_bfloat16 *orow = p.out + ((size_t)(tok0 + t) * p.num_q_heads + head) * D + 32 * i;
+    for (int i = 0; i < D / 32; ++i) tmem_ld32(trow + o_col + 32 * i, o[i]);
+    tmem_ld_wait();
+    tc_fence_before();
+    mbar_arrive(o_free);
+    const float inv = 1.f / l;
+    if (t < q_rows) {
+        __nv_bfloat16 *orow = p.out + ((size_t)(tok0 + t) * p.num_q_heads + head) * D;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-                w.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-                w.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-                w.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-                st16(orow + 8 * c, w);
+                w.x = pack_bf16x2(__uint_as_float(o[i][8 * c + 0]) * inv, __uint_as_float(o[i][8 * c + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(o[i][8 * c + 2]) * inv, __uint_as_float(o[i][8 * c + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(o[i][8 * c + 4]) * inv, __uint_as_float(o[i][8 * c + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(o[i][8 * c + 6]) * inv, __uint_as_float(o[i][8 * c + 7]) * inv);
+                st16(orow + 32 * i + 8 * c, w);
             }
         }
     }
 }
 
+// TMA descriptor of q as {D, Hq, T} (innermost first), boxes of
+// {64, 1, 128}: one 64-dim slab of 128 tokens of one head, 128-byte swizzle.
+struct PrefillMaps {
+    CUtensorMap q;
+};
+
+// Gathers staged tile blockIdx.x (K for blockIdx.y = 0, V for 1) from the
+// paged cache: 16-byte chunks, rows of one kv head's keys, swizzled as the
+// prefill kernel's shared-memory tiles.
 template <int D>
-__global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(256) stage_kernel(const __grid_constant__ PrefillParams p) {
+    constexpr int kRowChunks = D / 8;
+    const int kv = blockIdx.y;
+    const StageTile st = p.stages[blockIdx.x];
+    const int n = p.seq_lens[st.seq];
+    const int32_t *bt_row = p.block_tables + (size_t)st.seq * p.max_blocks_per_seq;
+    const __nv_bfloat16 *cache = kv ? p.v_cache : p.k_cache;
+    uint8_t *tile = p.staged + ((size_t)blockIdx.x * 2 + kv) * (128 * D * 2);
+    for (int c = threadIdx.x; c < 128 * kRowChunks; c += 256) {
+        const int row = c / kRowChunks, ch = c % kRowChunks;
+        const int key = 128 * st.tile + row;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (key < n) {
+            const int blk = __ldg(bt_row + (key >> 4));
+            v = ld_stream16(cache + (((size_t)blk * kBlockSize + (key & 15)) * p.num_kv_heads + st.kv_head) * D + ch * 8);
+        }
+        st16(tile + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4), v);
+    }
+}
+
+// One persistent CTA per SM works through its tiles [cta_start[c],
+// cta_start[c + 1]).  Barrier phases run on across tiles: the rings of K and
+// V stages, the per-step handshakes (S ready, P ready) and the per-tile ones
+// (Q loaded, Q free, O ready, O free).
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps maps) {
     using C = PrefillCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQA = smem_u32(smem + C::kQAOff);
     const uint32_t sQB = smem_u32(smem + C::kQBOff);
-    const uint32_t sKV = smem_u32(smem + C::kKVOff);
+    const uint32_t sK = smem_u32(smem + C::kKOff);
+    const uint32_t sV = smem_u32(smem + C::kVOff);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-    uint64_t *q_full = bars + 0;
-    uint64_t *kv_full = bars + 1;   // [2]
-    uint64_t *kv_empty = bars + 3;  // [2]: both heads' PV of the stage's tile are complete
-    uint64_t *sA_full = bars + 5, *sB_full = bars + 6;
-    uint64_t *pA_full = bars + 7, *pB_full = bars + 8;
-    uint64_t *oA_done = bars + 9, *oB_done = bars + 10;
+    uint64_t *q_full = bars + C::kBarQ, *q_empty = bars + C::kBarQEmpty;
+    uint64_t *k_full = bars + C::kBarKFull, *k_empty = bars + C::kBarKEmpty;
+    uint64_t *v_full = bars + C::kBarVFull, *v_empty = bars + C::kBarVEmpty;
+    uint64_t *sA_full = bars + C::kBarSA, *sB_full = bars + C::kBarSB;
+    uint64_t *pA_full = bars + C::kBarPA, *pB_full = bars + C::kBarPB;
+    uint64_t *oA_done = bars + C::kBarOA, *oB_done = bars + C::kBarOB;
+    uint64_t *oA_free = bars + C::kBarOAFree, *oB_free = bars + C::kBarOBFree;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kTmemSlotOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (blockIdx.x >= p.num_tiles) return;
-    const PrefillTile tile = p.tiles[blockIdx.x];
-    const int seq = tile.seq, q0 = tile.q_start;
-    const int hA = tile.head;
-    const bool two = tile.num_heads == 2;
-    const int hB = hA + 1;
-    const int tok0 = p.cu_seqlens_q[seq] + q0;
-    const int L = p.cu_seqlens_q[seq + 1] - p.cu_seqlens_q[seq];
-    const int n = p.seq_lens[seq];
-    const int q_rows = min(128, L - q0);
-    const int nkv = tile.n_kv_tiles;  // 128-key tiles covering keys 0 .. n - L + q0 + q_rows - 1
-    const int g = hA / p.group;
+    if (blockIdx.x >= p.num_ctas) return;
+    const int t_begin = p.cta_start[blockIdx.x], t_end = p.cta_start[blockIdx.x + 1];
+    if (t_begin >= t_end) return;
 
     if (tid == 0) {
-        mbar_init(q_full, C::kLoaders);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&kv_full[s], C::kLoaders);
-            mbar_init(&kv_empty[s], 1);
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < C::kKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::kVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         mbar_init(sA_full, 1);
         mbar_init(sB_full, 1);
@@ -298,6 +394,8 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
         mbar_init(pB_full, 128);
         mbar_init(oA_done, 1);
         mbar_init(oB_done, 1);
+        mbar_init(oA_free, 128);
+        mbar_init(oB_free, 128);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -310,174 +408,170 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     bool err = false;
 
-    if (warp == 0) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    if (warp < 4) {
+        warpgroup_reg_dealloc<C::kRegsLow>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            // The tensor pipe runs dry unless this thread issues an MMA
+            // every few dozen cycles while it shares its SM sub-partition
+            // with two softmax warps, so all descriptors are formed once:
+            // the start-address field holds address >> 4 in the low bits,
+            // so a byte offset o within shared memory adds o >> 4.
             constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, D, false, true);
-            auto mma_s = [&](uint32_t sQ, int j, uint32_t col) {
-                const uint32_t sK = sKV + (j & 1) * 2 * C::kTileBytes;
+            constexpr uint32_t kTileStep = C::kTileBytes >> 4;
+            const uint64_t dQA = umma_desc_sw128(sQA, 16, 1024), dQB = umma_desc_sw128(sQB, 16, 1024);
+            const uint64_t dK = umma_desc_sw128(sK, 16, 1024), dV = umma_desc_sw128(sV, 16384, 1024);
+            auto mma_s = [&](uint64_t dq, uint64_t dk, uint32_t col) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {  // 16 dims per MMA
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + col, umma_desc_sw128(sQ + off, 16, 1024),
-                                 umma_desc_sw128(sK + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                    umma_bf16_ss(tmem + col, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            auto mma_pv = [&](uint32_t p_col, int j, uint32_t o_col) {
-                const uint32_t sV = sKV + (j & 1) * 2 * C::kTileBytes + C::kTileBytes;
+            auto mma_pv = [&](uint64_t dv, uint32_t p_col, uint32_t o_col, uint32_t acc0) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)  // 16 keys per MMA; P: 8 columns of bf16 pairs
-                    umma_bf16_ts(tmem + o_col, tmem + p_col + 8 * kk, umma_desc_sw128(sV + kk * 2048, 16384, 1024),
-                                 idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + o_col, tmem + p_col + 8 * kk, dv + ((kk * 2048) >> 4), idesc_pv,
+                                 kk > 0 ? 1u : acc0);
             };
-            if (!err && !mbar_wait(q_full, 0)) err = true;
-            if (!err && !mbar_wait(&kv_full[0], 0)) err = true;
-            tc_fence_after();
-            mma_s(sQA, 0, C::kSA);
-            umma_commit(sA_full);
-            if (two) {
-                mma_s(sQB, 0, C::kSB);
-                umma_commit(sB_full);
-            }
-            for (int j = 0; j < nkv; ++j) {
-                const bool next = j + 1 < nkv;
-                if (!err && !mbar_wait(pA_full, j & 1)) err = true;
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                if (!err && !mbar_wait(bar, parity)) err = true;
+            };
+            int vs = 0, ks = 0;          // ring slots of the next V and K tiles
+            uint32_t vph = 0, kph = 0;   // and their phases
+            uint32_t itA = 0, itB = 0;   // 128-key steps of head A / head B so far
+            uint32_t kA = 0, kB = 0;     // tiles of head A / head B so far
+            for (int ti = t_begin; ti < t_end; ++ti) {
+                const PrefillTile tile = p.tiles[ti];
+                const bool two = tile.num_heads == 2;
+                const int nkv = tile.n_kv_tiles;
+                wait(q_full, (uint32_t)(ti - t_begin) & 1);
+                wait(&k_full[ks], kph);
                 tc_fence_after();
-                mma_pv(C::kSA, j, C::kOA);
-                if (!next) umma_commit(oA_done);
-                if (next) {
-                    if (!err && !mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) err = true;
-                    tc_fence_after();
-                    mma_s(sQA, j + 1, C::kSA);
-                    umma_commit(sA_full);
-                }
+                uint64_t dk = dK + ks * kTileStep;
+                mma_s(dQA, dk, C::kSA);
+                umma_commit(sA_full);
                 if (two) {
-                    if (!err && !mbar_wait(pB_full, j & 1)) err = true;
-                    tc_fence_after();
-                    mma_pv(C::kSB, j, C::kOB);
-                    if (!next) umma_commit(oB_done);
-                }
-                umma_commit(&kv_empty[j & 1]);
-                if (two && next) {
-                    mma_s(sQB, j + 1, C::kSB);
+                    mma_s(dQB, dk, C::kSB);
                     umma_commit(sB_full);
                 }
-            }
-            // nothing of ours may be in flight when TMEM is released
-            if (!err && !mbar_wait(&kv_empty[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1)) err = true;
-        }
-    } else if (warp < C::kSoftA) {
-        // ------------------------------------------------ loaders
-        // A warp copies whole 16-token blocks: its lanes' (row, chunk) pairs
-        // and their swizzled destinations are the same for every block.
-        constexpr int kPerLane = 16 * (D / 8) / 32;  // chunks per lane per block
-        const int lw = warp - 1;                     // loader warp 0..2
-        const int kv_stride = p.num_kv_heads * D;    // elements between tokens of a block
-        int src_col[kPerLane], row_of[kPerLane];
-        uint32_t dst_off[kPerLane];
-#pragma unroll
-        for (int k = 0; k < kPerLane; ++k) {
-            const int cidx = lane + 32 * k;
-            const int row = cidx / (D / 8), ch = cidx % (D / 8);
-            row_of[k] = row;
-            src_col[k] = 8 * ch;
-            dst_off[k] = (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        }
-        const int32_t *bt_row = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
-        // Q tiles: 16-row groups of both heads dealt out to the loader warps
-        {
-            const size_t q_stride = (size_t)p.num_q_heads * D;
-            for (int grp = lw; grp < (two ? 16 : 8); grp += C::kLoadWarps) {
-                const int hh = grp >> 3, r0 = 16 * (grp & 7);
-                const uint32_t sQ = hh ? sQB : sQA;
-                const __nv_bfloat16 *qh = p.q + (size_t)tok0 * q_stride + (size_t)(hh ? hB : hA) * D;
-#pragma unroll
-                for (int k = 0; k < kPerLane; ++k) {
-                    const int row = r0 + row_of[k];
-                    const uint32_t dst = sQ + r0 * 128 + dst_off[k];
-                    if (row < q_rows)
-                        cp_async16(dst, qh + (size_t)row * q_stride + src_col[k]);
-                    else
-                        st_shared_zero16(dst);
-                }
-            }
-        }
-        cp_async_commit();
-        // Tiles 0 and 1 go out at once; tile j >= 2 reuses the stage of tile
-        // j - 2 once both heads' PV of that tile is complete.  A tile's
-        // arrival is signalled before any wait on a stage, since the MMAs
-        // that free the stage depend on it.  The tile's 8 blocks (K and V)
-        // are dealt out to the loader warps.
-        auto issue_tile = [&](int j) {
-            const uint32_t sK = sKV + (j & 1) * 2 * C::kTileBytes, sV = sK + C::kTileBytes;
-            for (int b = lw; b < 8; b += C::kLoadWarps) {  // block within the tile
-                const int key0 = 128 * j + 16 * b;  // its first key
-                const uint32_t tile_off = 16 * b * 128;
-                if (key0 < n) {
-                    const int blk = __ldg(bt_row + (key0 >> 4));
-                    const size_t base = (size_t)blk * 16 * kv_stride + (size_t)g * D;
-                    const __nv_bfloat16 *kb = p.k_cache + base, *vb = p.v_cache + base;
-#pragma unroll
-                    for (int k = 0; k < kPerLane; ++k) {
-                        const int off = row_of[k] * kv_stride + src_col[k];
-                        if (key0 + row_of[k] < n) {
-                            cp_async16(sK + tile_off + dst_off[k], kb + off);
-                            cp_async16(sV + tile_off + dst_off[k], vb + off);
-                        } else {
-                            st_shared_zero16(sK + tile_off + dst_off[k]);
-                            st_shared_zero16(sV + tile_off + dst_off[k]);
+                umma_commit(&k_empty[ks]);
+                if (nkv == 1) umma_commit(q_empty);
+                if (++ks == C::kKStages) { ks = 0; kph ^= 1u; }
+                for (int j = 0; j < nkv; ++j) {
+                    const bool next = j + 1 < nkv;
+                    const uint64_t dv = dV + vs * kTileStep;
+                    const uint32_t acc0 = j > 0 ? 1u : 0u;
+                    wait(pA_full, itA & 1);
+                    if (j == 0 && kA > 0) wait(oA_free, (kA - 1) & 1);  // previous tile's O_A read out
+                    wait(&v_full[vs], vph);
+                    tc_fence_after();
+                    mma_pv(dv, C::kSA, C::kOA, acc0);
+                    if (!next) umma_commit(oA_done);
+                    if (next) {
+                        wait(&k_full[ks], kph);
+                        tc_fence_after();
+                        dk = dK + ks * kTileStep;
+                        mma_s(dQA, dk, C::kSA);
+                        umma_commit(sA_full);
+                    }
+                    if (two) {
+                        wait(pB_full, itB & 1);
+                        if (j == 0 && kB > 0) wait(oB_free, (kB - 1) & 1);
+                        tc_fence_after();
+                        mma_pv(dv, C::kSB, C::kOB, acc0);
+                        if (!next) umma_commit(oB_done);
+                    }
+                    umma_commit(&v_empty[vs]);
+                    if (next) {
+                        if (two) {
+                            mma_s(dQB, dk, C::kSB);
+                            umma_commit(sB_full);
                         }
+                        umma_commit(&k_empty[ks]);
+                        if (j + 2 == nkv) umma_commit(q_empty);  // last S of the tile issued
+                        if (++ks == C::kKStages) { ks = 0; kph ^= 1u; }
                     }
-                } else {
+                    if (++vs == C::kVStages) { vs = 0; vph ^= 1u; }
+                    ++itA;
+                    if (two) ++itB;
+                }
+                ++kA;
+                if (two) ++kB;
+            }
+            // nothing of ours may be in flight when TMEM is released: the
+            // last commit on v_empty covers every MMA issued
+            const int last_v = vs == 0 ? C::kVStages - 1 : vs - 1;
+            wait(&v_empty[last_v], vs == 0 ? vph ^ 1u : vph);
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------------------------ loads
+            int vs = 0, ks = 0;
+            uint32_t vuse = 0, kuse = 0;  // K / V tiles loaded so far
+            for (int ti = t_begin; ti < t_end; ++ti) {
+                const PrefillTile tile = p.tiles[ti];
+                const bool two = tile.num_heads == 2;
+                const int nkv = tile.n_kv_tiles;
+                const int hA = tile.head;
+                const int tok0 = p.cu_seqlens_q[tile.seq] + tile.q_start;
+                if (ti > t_begin && !err && !mbar_wait(q_empty, (uint32_t)(ti - t_begin - 1) & 1)) err = true;
+                mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kTileBytes);
 #pragma unroll
-                    for (int k = 0; k < kPerLane; ++k) {
-                        st_shared_zero16(sK + tile_off + dst_off[k]);
-                        st_shared_zero16(sV + tile_off + dst_off[k]);
-                    }
+                for (int s = 0; s < C::kSlabs; ++s) {
+                    tma_load_3d(sQA + s * 16384, &maps.q, q_full, 64 * s, hA, tok0);
+                    if (two) tma_load_3d(sQB + s * 16384, &maps.q, q_full, 64 * s, hA + 1, tok0);
+                }
+                // staged tile kv_base + j: K then V, kTileBytes each
+                const uint8_t *kv_tiles = p.staged + (size_t)tile.kv_base * 2 * C::kTileBytes;
+                auto load_k = [&](int j) {
+                    if (kuse >= (uint32_t)C::kKStages && !err &&
+                        !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1))
+                        err = true;
+                    mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
+                    bulk_load(sK + ks * C::kTileBytes, kv_tiles + (size_t)j * 2 * C::kTileBytes, C::kTileBytes,
+                              &k_full[ks]);
+                    ++kuse;
+                    if (++ks == C::kKStages) ks = 0;
+                };
+                auto load_v = [&](int j) {
+                    if (vuse >= (uint32_t)C::kVStages && !err &&
+                        !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1))
+                        err = true;
+                    mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
+                    bulk_load(sV + vs * C::kTileBytes, kv_tiles + ((size_t)j * 2 + 1) * C::kTileBytes, C::kTileBytes,
+                              &v_full[vs]);
+                    ++vuse;
+                    if (++vs == C::kVStages) vs = 0;
+                };
+                load_k(0);
+                for (int j = 0; j < nkv; ++j) {
+                    if (j + 1 < nkv) load_k(j + 1);
+                    load_v(j);
                 }
             }
-            cp_async_commit();
-        };
-        issue_tile(0);
-        if (nkv >= 2) {
-            issue_tile(1);
-            cp_async_wait<2>();  // Q has landed
-        } else {
-            cp_async_wait<1>();
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(q_full);
-        if (nkv >= 2)
-            cp_async_wait<1>();  // tile 0 has landed
-        else
-            cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(&kv_full[0]);
-        for (int j = 2; j < nkv; ++j) {
-            cp_async_wait<0>();  // tile j - 1 has landed
-            fence_proxy_async_smem();
-            mbar_arrive(&kv_full[(j - 1) & 1]);
-            if (!err && !mbar_wait(&kv_empty[j & 1], ((j - 2) >> 1) & 1)) err = true;
-            issue_tile(j);
-        }
-        if (nkv >= 2) {
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            mbar_arrive(&kv_full[(nkv - 1) & 1]);
         }
     } else {
         // ------------------------------------------------ softmax warps
+        warpgroup_reg_alloc<C::kRegsHigh>();
         const bool headA = warp < C::kSoftB;
-        if (headA || two) {
-            const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-            const int t = quarter * 32 + lane;
-            const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+        const int t = quarter * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint32_t it = 0, k = 0;
+        for (int ti = t_begin; ti < t_end; ++ti) {
+            const PrefillTile tile = p.tiles[ti];
+            if (!headA && tile.num_heads != 2) continue;
+            const int seq = tile.seq, q0 = tile.q_start;
+            const int tok0 = p.cu_seqlens_q[seq] + q0;
+            const int L = p.cu_seqlens_q[seq + 1] - p.cu_seqlens_q[seq];
+            const int n = p.seq_lens[seq];
+            const int q_rows = min(128, L - q0);
             const int first_pos = n - L + q0;
             const int pos = t < q_rows ? first_pos + t : 0;  // padding rows see key 0 only
-            softmax_head<D>(p, trow, headA ? C::kSA : C::kSB, headA ? C::kOA : C::kOB, headA ? sA_full : sB_full,
-                            headA ? pA_full : pB_full, headA ? oA_done : oB_done, nkv, t, q_rows, pos, first_pos,
-                            tok0, headA ? hA : hB, err);
+            softmax_tile<D>(p, trow, headA ? C::kSA : C::kSB, headA ? C::kOA : C::kOB, headA ? sA_full : sB_full,
+                            headA ? pA_full : pB_full, headA ? oA_done : oB_done, headA ? oA_free : oB_free,
+                            tile.n_kv_tiles, it, k, t, q_rows, pos, first_pos, tok0, tile.head + (headA ? 0 : 1), err);
+            ++k;
         }
     }
     if (err) atomicOr(p.status, kStatusWaitTimeout);
@@ -487,9 +581,47 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
     if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on the driver library).
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn tensor_map_encoder() {
+    static std::atomic<EncodeFn> fn{nullptr};
+    EncodeFn f = fn.load(std::memory_order_acquire);
+    if (f) return f;
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !ptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    f = reinterpret_cast<EncodeFn>(ptr);
+    fn.store(f, std::memory_order_release);
+    return f;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle.
+bool encode_bf16(EncodeFn enc, CUtensorMap *map, const void *base, int rank, const cuuint64_t *dims,
+                 const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides_bytes, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     using C = PrefillCfg<D>;
+    EncodeFn enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    PrefillMaps maps;
+    const cuuint64_t dims[3] = {D, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.num_tokens};
+    const cuuint64_t strides[2] = {D * 2ull, (cuuint64_t)p.num_q_heads * D * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if (!encode_bf16(enc, &maps.q, p.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
     static std::atomic<uint64_t> configured{0};  // one bit per device
     int dev = 0;
     cudaGetDevice(&dev);
@@ -500,7 +632,8 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    prefill_kernel<D><<<p.num_tiles, C::kThreads, C::kSmemBytes, stream>>>(p);
+    stage_kernel<D><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
+    prefill_kernel<D><<<p.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(p, maps);
     return cudaGetLastError();
 }
 

@@ -84,6 +84,13 @@ def test_plan_invariants(lib, name):
     G = lay.num_q_heads // lay.num_kv_heads
     assert info["workspace_bytes"] >= info["table_bytes"] + info["num_partials"] * G * lay.head_dim * 4
     assert plan.workspace_bytes == info["workspace_bytes"]
+    # prefill tiles are dealt to at most one persistent CTA per SM; K/V of
+    # every prefill segment are staged per kv head in 128-key tiles
+    assert info["num_prefill_ctas"] == min(info["num_prefill_tiles"], info["num_sms"])
+    pre = ql > 16 if prefill_on_tensor_cores else np.zeros_like(ql, dtype=bool)
+    staged = int(sum(-(-n // 128) for n in sl[pre])) * lay.num_kv_heads
+    assert info["num_staged_kv_tiles"] == staged
+    assert info["workspace_bytes"] >= staged * 2 * 128 * lay.head_dim * 2
 
 
 def test_plan_rebuild_in_place(lib):
