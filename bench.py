@@ -407,9 +407,9 @@ def run_ours(args):
         return [t.elapsed_ms() for t in trs]
 
     dec_ms = statistics.mean(s["decode"] for s in traced_pass(("decode",)))
-    other = traced_pass(("table_copy", "combine", "prefill"))
+    other = traced_pass(("plan_wait", "combine", "prefill"))
     comb_ms = statistics.mean(s["combine"] for s in other)
-    copy_ms = statistics.mean(s["table_copy"] for s in other)
+    wait_ms = statistics.mean(s["plan_wait"] for s in other)
     prefill_ms = statistics.mean(s["prefill"] for s in other)
     split = decode_prefill_split(lay)
     roofline_decode = roofline_prefill = None
@@ -449,7 +449,8 @@ def run_ours(args):
                  ("bt", bt), ("cu", cu), ("sl", sl))}
         dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
         out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        h2d = sum(x.numel() * x.element_size() for x in host.values())
+        # inputs, plus the plan tables each step's build uploads
+        h2d = sum(x.numel() * x.element_size() for x in host.values()) + info["table_bytes"]
         d2h = out_host.numel() * out_host.element_size()
         e_ms = []
         for i in range(args.warmup + args.steps):
@@ -497,7 +498,7 @@ def run_ours(args):
                        "tokens_per_step": lay.num_tokens,
                        "l2": "flushed before every timed step (1 GiB write, outside the events)",
                        "plan_us_host": 1e6 * statistics.median(plan_times),
-                       "stages_ms": {"table_copy": copy_ms, "decode": dec_ms, "combine": comb_ms,
+                       "stages_ms": {"plan_wait": wait_ms, "decode": dec_ms, "combine": comb_ms,
                                      "prefill": prefill_ms,
                                      "note": "separate traced passes; event records add GPU time"},
                        "parallelism": f"replicas x{world} (weak: one batch per GPU)",

@@ -99,31 +99,40 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
                          void *stream);
 
 /*
- * Work partition for pa_attention_varlen (host only; queues no GPU work).
- * From the host copies of cu_seqlens_q and seq_lens (the same values the
+ * Work partition for pa_attention_varlen.  From the host copies of cu_seqlens_q and seq_lens (the same values the
  * device arrays will hold) it splits the step into balanced GPU work:
  * segments with q_len <= 16 (decodes, speculative-verification shapes) are
  * cut into equal runs of 16-token KV blocks over all query rows and kv heads
  * (split-KV), one run per CTA and SM, the partials of rows cut between runs
  * being merged by the last CTA to finish them; longer segments are cut into
  * 128-query tiles for pairs of query heads sharing a kv head, for the
- * tensor-core prefill kernel, longest tiles first.
+ * tensor-core prefill kernel and dealt to at most one CTA per SM.  The
+ * resulting tables are uploaded to device memory the plan owns, on a stream
+ * of the plan's own (an asynchronous copy from page-locked memory; the only
+ * GPU work a build queues).
  *   h_cu_seqlens_q  host [S+1] int32
  *   h_seq_lens      host [S] int32
  *   dims            host; T, S, Hq, Hkv, D, B are used
- *   device          CUDA device ordinal the plan is sized for (its SM count
- *                   is read once per process and cached; -1 = assume 148 SMs)
+ *   device          CUDA device ordinal the plan is built for (its SM count
+ *                   is read once per process and cached; the device tables
+ *                   are allocated there).  -1 builds a host-only plan that
+ *                   assumes 148 SMs, for inspection with pa_plan_get_info;
+ *                   attention calls reject it (PA_ERR_PLAN).
  *   out             in/out.  If *out is NULL a new plan is created and
  *                   stored there; the caller owns it and frees it with
  *                   pa_plan_destroy.  If *out holds a plan from an earlier
  *                   call (same device), that plan is rebuilt in place and its
- *                   host buffers are reused, so that a caller rebuilding one
- *                   plan per step allocates nothing after the first step.
- *                   The plan's tables live in page-locked host memory and are
- *                   copied into the workspace by every attention call that
- *                   uses the plan; rebuilding or destroying a plan first waits
- *                   until the most recent such copy has executed.  A plan may
- *                   serve every layer of a step and several streams.
+ *                   buffers are reused (grown when too small), so that a
+ *                   caller rebuilding one plan per step allocates nothing
+ *                   after the first steps.  Rebuilding or destroying a plan
+ *                   first waits (on the host) until its last upload and the
+ *                   last attention call that used it have finished on the
+ *                   GPU, so an engine that builds step k+1's plan while step
+ *                   k runs keeps two plans and alternates.  A plan may serve
+ *                   every layer of a step; calls that use the same plan must
+ *                   not overlap on the GPU (queue them on one stream, or
+ *                   order them with events), because the merge tickets of
+ *                   split rows live in the plan's device tables.
  * On error a plan passed in *out is left unusable for attention calls until
  * it is rebuilt successfully; it must still be destroyed.
  * Errors: PA_ERR_NULL, PA_ERR_SHAPE (cu_seqlens not starting at 0, not
@@ -155,9 +164,8 @@ int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
  * (0 for a NULL plan).  256-byte alignment of the workspace is required. */
 size_t pa_plan_workspace_bytes(const pa_plan *plan);
 
-/* Frees a plan (NULL is allowed), after waiting until the table copy of the
- * most recent attention call that used it has executed.  Work queued with it
- * is not affected. */
+/* Frees a plan (NULL is allowed), after waiting until its last upload and
+ * the last attention call that used it have finished on the GPU. */
 void pa_plan_destroy(pa_plan *plan);
 
 /*
@@ -182,9 +190,15 @@ void pa_plan_destroy(pa_plan *plan);
  *   d_out           device [T][Hq][D] bf16, written
  *   plan            from pa_plan_build with the same dims
  *   d_workspace     device scratch of pa_plan_workspace_bytes(plan) bytes,
- *                   256-byte aligned; the plan tables are copied into it on
- *                   `stream` and the split partials live there.  Two calls
+ *                   256-byte aligned: a status word (zero-fill it before
+ *                   first use), then scratch with no initial value (split
+ *                   partials, staged K/V tiles of prefill segments).  Calls
+ *                   with different plans may share a workspace.  Two calls
  *                   in flight at once need two workspaces.
+ * After a call that reported an error, rebuild the plan (its merge tickets
+ * may be left taken) and reset the workspace's status word.
+ * The call makes `stream` wait for the plan's upload, then queues its
+ * kernels; nothing is copied from the host.
  * Errors: PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_UNSUPPORTED,
  * PA_ERR_PLAN, PA_ERR_WORKSPACE, PA_ERR_CUDA.
  */
@@ -199,9 +213,11 @@ int pa_attention_varlen(const void *d_q, const void *d_k_cache, const void *d_v_
  * non-NULL entry of trace->events (a cudaEvent_t created by the caller) is
  * recorded on `stream` at a fixed point of the call, so that the caller can
  * time every kernel on the stream it runs on:
- *   [0] before the plan-table copy     [1] before the split-KV decode kernel
- *   [2] after the split-KV kernel      [3] after the combine kernel
- *   [4] before the prefill kernel      [5] after the prefill kernel
+ *   [0] before the wait for the plan's upload
+ *   [1] before the split-KV decode kernel (which also merges split rows)
+ *   [2] after the split-KV kernel      [3] = [2] (no separate combine kernel)
+ *   [4] before the K/V staging and prefill kernels
+ *   [5] after the prefill kernel
  * Events of stages that do not run are still recorded (adjacent), so every
  * interval is defined.  Results are identical to pa_attention_varlen.
  */
@@ -215,13 +231,21 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
                            size_t workspace_bytes, void *stream, const pa_trace *trace);
 
 /*
- * Status word of a workspace after a pa_attention_varlen call: waits for
- * `stream`, then copies the word to *status.  0 means no error; bit 0 means
- * some wait inside a kernel gave up after about a second (the kernels never
- * block longer, and the affected outputs are undefined).  The word is reset
- * by every call that uses the workspace.
+ * Status word of a workspace: waits for `stream`, then copies the word to
+ * *status.  0 means no error; bit 0 means some wait inside a kernel gave up
+ * after about a second (the kernels never block longer, and the affected
+ * outputs are undefined).  Error bits accumulate over the calls that used
+ * the workspace until pa_workspace_reset clears them.
  */
 int pa_workspace_status(const void *d_workspace, void *stream, uint32_t *status);
+
+/*
+ * Zeroes the status word of a workspace (a memset queued on `stream`);
+ * `plan` is any plan the workspace serves.  Needed only after a call whose
+ * status reported an error.
+ * Errors: PA_ERR_NULL, PA_ERR_WORKSPACE (not 256-byte aligned), PA_ERR_CUDA.
+ */
+int pa_workspace_reset(void *d_workspace, const pa_plan *plan, void *stream);
 
 /*
  * Opt-in check of the data-dependent preconditions, on the device, then a
@@ -262,12 +286,14 @@ int pa_validate_inputs(const int64_t *d_slot_mapping, const int32_t *d_block_tab
  *     that first call before any stream capture.  A failed lookup returns
  *     PA_ERR_CUDA.
  *   - All calls on a device share the one array, which keeps the last call's
- *     contents.  Nothing in it needs to start at zero: every call first
- *     copies its plan's tables over the front of it and writes each partial
- *     result before reading it.  Calls whose GPU work overlaps in time (two
- *     streams, or two threads' streams) race on the array and give undefined
- *     results; order them, or use pa_attention_varlen with separate
- *     workspaces.
+ *     contents.  Its first word is a status word like a workspace's (zero
+ *     at load; the kernels only ever set error bits in it, and its address
+ *     is not exposed, so it is not read or cleared).  The rest is scratch
+ *     that every call writes before reading; the plan's tables live with
+ *     the plan.  Calls
+ *     whose GPU work overlaps in time (two streams, or two threads' streams)
+ *     race on the array and give undefined results; order them, or use
+ *     pa_attention_varlen with separate workspaces.
  */
 size_t pa_noalloc_scratch_bytes(void);
 int pa_attention_varlen_noalloc(const void *d_q, const void *d_k_cache, const void *d_v_cache,

@@ -94,6 +94,7 @@ def load_library():
             "pa_attention_varlen_noalloc": (I, [P, P, P, P, P, P, F, P, DP, P, P]),
             "pa_noalloc_scratch_bytes": (SZ, []),
             "pa_workspace_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+            "pa_workspace_reset": (I, [P, P, P]),
             "pa_validate_scratch_bytes": (SZ, [DP]),
             "pa_validate_inputs": (I, [P, P, P, P, DP, P, SZ, P]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -226,8 +227,9 @@ class Plan:
 
 
 def workspace_for(plan: Plan, device=None) -> torch.Tensor:
-    """A device workspace of the size a plan needs (256-byte aligned by torch)."""
-    return torch.empty(max(plan.workspace_bytes, 1), dtype=torch.uint8,
+    """A zero-filled device workspace of the size a plan needs (256-byte
+    aligned by torch)."""
+    return torch.zeros(max(plan.workspace_bytes, 1), dtype=torch.uint8,
                        device=device if device is not None else "cuda")
 
 
@@ -235,9 +237,9 @@ class Trace(ctypes.Structure):
     """Events recorded around the kernels of one attention call (pa_trace)."""
     _fields_ = [("events", ctypes.c_void_p * 6)]
 
-    MARKS = {"table_copy": (0, 1), "decode": (1, 2), "combine": (2, 3), "prefill": (4, 5)}
+    MARKS = {"plan_wait": (0, 1), "decode": (1, 2), "combine": (2, 3), "prefill": (4, 5)}
 
-    def __init__(self, stages=("table_copy", "decode", "combine", "prefill")):
+    def __init__(self, stages=("plan_wait", "decode", "combine", "prefill")):
         """Record only the marks the named stages need (each record costs a
         couple of microseconds of GPU time)."""
         super().__init__()
@@ -293,12 +295,18 @@ def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, 
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:
-    """Error bits the last attention call left in a workspace (0 = none);
-    waits for the stream."""
+    """Error bits the attention calls since the last reset left in a
+    workspace (0 = none); waits for the stream."""
     st = ctypes.c_uint32(0)
     _check(load_library().pa_workspace_status(_dev_ptr(workspace, "workspace"), _stream_ptr(stream),
                                               ctypes.byref(st)), "pa_workspace_status")
     return int(st.value)
+
+
+def workspace_reset(workspace: torch.Tensor, plan: "Plan", stream=None) -> None:
+    """Zero a workspace's status word and merge tickets (after an error)."""
+    _check(load_library().pa_workspace_reset(_dev_ptr(workspace, "workspace"), plan.handle, _stream_ptr(stream)),
+           "pa_workspace_reset")
 
 
 def noalloc_scratch_bytes() -> int:

@@ -133,23 +133,19 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return PA_ERR_ALIGN;
     const WorkspaceLayout &w = plan->ws;
-    if (w.total > 0) {
-        if (!workspace || workspace_bytes < w.total) return PA_ERR_WORKSPACE;
-        if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
-    }
+    const TableLayout &tl = plan->tl;
+    if (!workspace || workspace_bytes < w.total) return PA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
+    // the plan's tables live on its device
+    int cur = -1;
+    if (!plan->d_tables || cudaGetDevice(&cur) != cudaSuccess || cur != plan->device) return PA_ERR_PLAN;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const uint8_t *tb = static_cast<const uint8_t *>(plan->d_tables);
     if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
-    if (w.table_bytes > 0) {
-        // Page-locked source: the copy runs in stream order without blocking
-        // the host; the plan's event marks when its buffer may be reused.
-        if (cudaMemcpyAsync(ws, plan->tables, w.table_bytes, cudaMemcpyHostToDevice, stream) !=
-            cudaSuccess)
-            return PA_ERR_CUDA;
-        if (plan->upload_event &&
-            cudaEventRecord(static_cast<cudaEvent_t>(plan->upload_event), stream) != cudaSuccess)
-            return PA_ERR_CUDA;
-    }
+    // the upload queued by the plan's build (usually long done)
+    if (cudaStreamWaitEvent(stream, static_cast<cudaEvent_t>(plan->upload_event), 0) != cudaSuccess)
+        return PA_ERR_CUDA;
     const float scale_log2 = scale * kLog2e;
     if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
     if (plan->num_units > 0) {
@@ -161,9 +157,10 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.out = static_cast<__nv_bfloat16 *>(out);
         p.partial_o = reinterpret_cast<float *>(ws + w.partial_o);
         p.partial_ml = reinterpret_cast<float2 *>(ws + w.partial_ml);
-        p.units = reinterpret_cast<const DecodeUnit *>(ws + w.units);
-        p.rows = reinterpret_cast<const DecodeRow *>(ws + w.rows);
-        p.combine = reinterpret_cast<CombineRow *>(ws + w.combine);
+        p.units = reinterpret_cast<const DecodeUnit *>(tb + tl.units);
+        p.rows = reinterpret_cast<const DecodeRow *>(tb + tl.rows);
+        p.combine = reinterpret_cast<const CombineRow *>(tb + tl.combine);
+        p.arrived = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(plan->d_tables) + tl.arrived);
         p.status = reinterpret_cast<uint32_t *>(ws + w.header);
         p.num_units = plan->num_units;
         p.num_q_heads = d.num_q_heads;
@@ -186,10 +183,10 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         pp.cu_seqlens_q = cu_seqlens_q;
         pp.seq_lens = seq_lens;
         pp.out = static_cast<__nv_bfloat16 *>(out);
-        pp.tiles = reinterpret_cast<const PrefillTile *>(ws + w.tiles);
-        pp.cta_start = reinterpret_cast<const int32_t *>(ws + w.cta_start);
+        pp.tiles = reinterpret_cast<const PrefillTile *>(tb + tl.tiles);
+        pp.cta_start = reinterpret_cast<const int32_t *>(tb + tl.cta_start);
         pp.num_ctas = plan->num_prefill_ctas;
-        pp.stages = reinterpret_cast<const StageTile *>(ws + w.stages);
+        pp.stages = reinterpret_cast<const StageTile *>(tb + tl.stages);
         pp.staged = ws + w.staged;
         pp.num_stages = plan->num_stages;
         pp.status = reinterpret_cast<uint32_t *>(ws + w.header);
@@ -204,6 +201,16 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
     }
     if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;
+    // the plan's next build waits for this
+    if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+extern "C" int pa_workspace_reset(void *workspace, const pa_plan *plan, void *stream_) {
+    if (!workspace || !plan) return PA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream_)) != cudaSuccess)
+        return PA_ERR_CUDA;
     return PA_OK;
 }
 

@@ -304,6 +304,15 @@ struct LoadCursor {
     bool done;
 };
 
+__device__ __forceinline__ void cursor_set_row(const DecodeParams &p, const DecodeUnit &end, LoadCursor &c,
+                                               int seq, int n_keys) {
+    c.bt_row = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
+    c.nblk = (n_keys + 15) >> 4;
+    c.bend = (c.r == end.row) ? end.block : c.nblk;
+    c.g = c.r % p.num_kv_heads;
+    c.bt_base = -1;
+}
+
 __device__ __forceinline__ void cursor_enter_row(const DecodeParams &p, const DecodeUnit &end,
                                                  LoadCursor &c) {
     if (c.r > end.row || (c.r == end.row && end.block == 0)) {
@@ -311,11 +320,7 @@ __device__ __forceinline__ void cursor_enter_row(const DecodeParams &p, const De
         return;
     }
     const DecodeRow row = p.rows[c.r];
-    c.bt_row = p.block_tables + (size_t)row.seq * p.max_blocks_per_seq;
-    c.nblk = (row.n_keys + 15) >> 4;
-    c.bend = (c.r == end.row) ? end.block : c.nblk;
-    c.g = c.r % p.num_kv_heads;
-    c.bt_base = -1;
+    cursor_set_row(p, end, c, row.seq, row.n_keys);
 }
 
 __device__ __forceinline__ int cursor_block_id(LoadCursor &c, int b, int lane) {
@@ -408,11 +413,13 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
     // Load cursor: this warp's next step to copy; S-1 steps run ahead.
     LoadCursor lc;
     {
+        // the unit carries its first row's segment and length: the first
+        // copies need no read of the row table
         const DecodeUnit st = p.units[unit];
         lc.r = st.row;
         lc.b = st.block;
-        lc.done = false;
-        cursor_enter_row(p, run_end, lc);
+        lc.done = st.row > run_end.row || (st.row == run_end.row && st.block >= run_end.block);
+        if (!lc.done) cursor_set_row(p, run_end, lc, st.seq, st.n_keys);
     }
 #pragma unroll
     for (int j = 0; j < S - 1; ++j) {
@@ -512,14 +519,14 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
             __threadfence();
             __syncwarp();
             int last = 0;
-            if (lane == 0) {
-                const CombineRow c = p.combine[row.combine];
-                last = atomicAdd(&p.combine[row.combine].arrived, 1) == c.piece_count - 1;
-            }
+            const CombineRow c = p.combine[row.combine];
+            if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.piece_count - 1;
             last = __shfl_sync(kFullMask, last, 0);
             if (last) {
                 __threadfence();
-                merge_split_row<D>(p, p.combine[row.combine], row.token, h0, lane, 32);
+                merge_split_row<D>(p, c, row.token, h0, lane, 32);
+                // every ticket of this call is taken: leave the counter at zero
+                if (lane == 0) p.arrived[row.combine] = 0u;
             }
         }
     });

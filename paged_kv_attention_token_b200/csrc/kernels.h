@@ -19,8 +19,9 @@ struct DecodeParams {
     float2 *partial_ml;     // [pieces][G]: (max in log2 units, sum)
     const DecodeUnit *units;
     const DecodeRow *rows;
-    CombineRow *combine;        // tickets live here; zero at upload
-    uint32_t *status;           // workspace status word (error bits), zero at upload
+    const CombineRow *combine;
+    uint32_t *arrived;          // per combine row: tickets taken (plan tables; zero between calls)
+    uint32_t *status;           // workspace status word (error bits)
     int num_units;
     int num_q_heads;
     int num_kv_heads;

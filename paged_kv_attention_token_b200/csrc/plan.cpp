@@ -44,9 +44,27 @@ constexpr int64_t kTileOverheadSteps = 2;
 // q, the final write or merge) stay small against the streaming.
 constexpr int64_t kMinBlocksPerUnit = 4;
 
-// Waits until the last table copy queued from this plan has executed.
-void wait_upload(const pa_plan *p) {
+// Scoped switch to the plan's device (plans own device memory, a stream and
+// events, which belong to the device they were made on).
+struct DeviceScope {
+    int prev = -1;
+    explicit DeviceScope(int device) {
+        if (device < 0) return;
+        cudaGetDevice(&prev);
+        if (prev != device) cudaSetDevice(device);
+    }
+    ~DeviceScope() {
+        int cur = -1;
+        cudaGetDevice(&cur);
+        if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+// Waits until the plan's last upload has executed and the last attention
+// call that read its tables has finished.
+void wait_idle(const pa_plan *p) {
     if (p->upload_event) cudaEventSynchronize(static_cast<cudaEvent_t>(p->upload_event));
+    if (p->use_event) cudaEventSynchronize(static_cast<cudaEvent_t>(p->use_event));
 }
 
 void free_tables(pa_plan *p) {
@@ -87,17 +105,47 @@ bool reserve_tables(pa_plan *p, size_t bytes) {
     return true;
 }
 
-void create_event(pa_plan *p) {
-    if (p->upload_event || p->device < 0) return;
-    int prev = -1;
-    cudaGetDevice(&prev);
-    if (prev != p->device) cudaSetDevice(p->device);
-    cudaEvent_t e = nullptr;
-    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess)
-        p->upload_event = e;
-    else
-        cudaGetLastError();
-    if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
+// Stream and events of a plan with a device (created once).
+bool create_sync_objects(pa_plan *p) {
+    if (p->device < 0) return true;
+    if (p->upload_stream && p->upload_event && p->use_event) return true;
+    DeviceScope scope(p->device);
+    if (!p->upload_stream) {
+        cudaStream_t s = nullptr;
+        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
+        p->upload_stream = s;
+    }
+    for (void **slot : {&p->upload_event, &p->use_event}) {
+        if (*slot) continue;
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+        *slot = e;
+    }
+    return true;
+}
+
+// Copies the host image of the tables to the plan's device buffer on the
+// plan's stream (the caller has waited for the plan to be idle).
+bool upload_tables(pa_plan *p) {
+    if (p->device < 0) return true;
+    DeviceScope scope(p->device);
+    const size_t bytes = p->tl.bytes;
+    if (p->d_capacity < bytes) {
+        if (p->d_tables) cudaFree(p->d_tables);
+        p->d_tables = nullptr;
+        p->d_capacity = 0;
+        const size_t cap = std::max<size_t>(bytes, 4096);
+        void *d = nullptr;
+        if (cudaMalloc(&d, cap) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        p->d_tables = d;
+        p->d_capacity = cap;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(p->upload_stream);
+    if (cudaMemcpyAsync(p->d_tables, p->tables, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return false;
+    return cudaEventRecord(static_cast<cudaEvent_t>(p->upload_event), s) == cudaSuccess;
 }
 
 int check_dims(const pa_dims *d) {
@@ -137,7 +185,11 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
         p = new (std::nothrow) pa_plan();
         if (!p) return PA_ERR_CUDA;
         p->device = device;
-        create_event(p);
+        if (!create_sync_objects(p)) {
+            cudaGetLastError();
+            pa_plan_destroy(p);
+            return PA_ERR_CUDA;
+        }
     } else if (p->device != device) {
         return PA_ERR_PLAN;
     }
@@ -221,9 +273,10 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
             const int64_t f = P ? total * u / P : 0;
             ustart[u] = f;
             while (r < R && prefix[r + 1] <= f) ++r;  // row holding block f
-            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)])};
+            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)]), r < R ? rows[r].seq : 0,
+                        r < R ? rows[r].n_keys : 0};
         }
-        units[P] = {(int32_t)R, 0};
+        units[P] = {(int32_t)R, 0, 0, 0};
     }
     // Pieces: a row is split if its blocks span more than one unit.
     std::vector<pa::CombineRow> combine;
@@ -253,16 +306,20 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     p->num_prefill_ctas = grid;
     p->num_stages = (int32_t)stages.size();
 
-    pa::WorkspaceLayout &w = p->ws;
+    pa::TableLayout &t = p->tl;
     size_t off = 0;
-    w.header = off;  off = pa::kHeaderBytes;
-    w.units = off;   off = align_up(off + sizeof(pa::DecodeUnit) * units.size(), pa::kWorkspaceAlign);
-    w.rows = off;    off = align_up(off + sizeof(pa::DecodeRow) * rows.size(), pa::kWorkspaceAlign);
-    w.combine = off; off = align_up(off + sizeof(pa::CombineRow) * combine.size(), pa::kWorkspaceAlign);
-    w.tiles = off;   off = align_up(off + sizeof(pa::PrefillTile) * tiles.size(), pa::kWorkspaceAlign);
-    w.cta_start = off; off = align_up(off + sizeof(int32_t) * cta_start.size(), pa::kWorkspaceAlign);
-    w.stages = off;  off = align_up(off + sizeof(pa::StageTile) * stages.size(), pa::kWorkspaceAlign);
-    w.table_bytes = off;
+    t.units = off;     off = align_up(off + sizeof(pa::DecodeUnit) * units.size(), pa::kWorkspaceAlign);
+    t.rows = off;      off = align_up(off + sizeof(pa::DecodeRow) * rows.size(), pa::kWorkspaceAlign);
+    t.combine = off;   off = align_up(off + sizeof(pa::CombineRow) * combine.size(), pa::kWorkspaceAlign);
+    t.tiles = off;     off = align_up(off + sizeof(pa::PrefillTile) * tiles.size(), pa::kWorkspaceAlign);
+    t.cta_start = off; off = align_up(off + sizeof(int32_t) * cta_start.size(), pa::kWorkspaceAlign);
+    t.stages = off;    off = align_up(off + sizeof(pa::StageTile) * stages.size(), pa::kWorkspaceAlign);
+    t.arrived = off;   off = align_up(off + sizeof(uint32_t) * combine.size(), pa::kWorkspaceAlign);
+    t.bytes = off;
+
+    pa::WorkspaceLayout &w = p->ws;
+    off = 0;
+    w.header = off;    off = pa::kHeaderBytes;
     w.partial_o = off;
     off = align_up(off + sizeof(float) * (size_t)piece_base * p->group * d.head_dim, pa::kWorkspaceAlign);
     w.partial_ml = off;
@@ -272,22 +329,30 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     off += stages.size() * 2 * (size_t)pa::kPrefillTileN * d.head_dim * 2;
     w.total = align_up(off, pa::kWorkspaceAlign);
 
-    wait_upload(p);  // the previous build's tables may still be in a queued copy
-    if (!reserve_tables(p, w.table_bytes)) {
+    {
+        DeviceScope scope(p->device);
+        wait_idle(p);  // no queued copy reads the host image, no kernel the device tables
+    }
+    if (!reserve_tables(p, t.bytes)) {
         if (fresh) pa_plan_destroy(p);
         return PA_ERR_CUDA;
     }
-    std::memset(p->tables, 0, w.table_bytes);
-    std::memcpy(p->tables + w.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
+    std::memset(p->tables, 0, t.bytes);
+    std::memcpy(p->tables + t.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
     if (!rows.empty())
-        std::memcpy(p->tables + w.rows, rows.data(), sizeof(pa::DecodeRow) * rows.size());
+        std::memcpy(p->tables + t.rows, rows.data(), sizeof(pa::DecodeRow) * rows.size());
     if (!combine.empty())
-        std::memcpy(p->tables + w.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
+        std::memcpy(p->tables + t.combine, combine.data(), sizeof(pa::CombineRow) * combine.size());
     if (!tiles.empty())
-        std::memcpy(p->tables + w.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
-    std::memcpy(p->tables + w.cta_start, cta_start.data(), sizeof(int32_t) * cta_start.size());
+        std::memcpy(p->tables + t.tiles, tiles.data(), sizeof(pa::PrefillTile) * tiles.size());
+    std::memcpy(p->tables + t.cta_start, cta_start.data(), sizeof(int32_t) * cta_start.size());
     if (!stages.empty())
-        std::memcpy(p->tables + w.stages, stages.data(), sizeof(pa::StageTile) * stages.size());
+        std::memcpy(p->tables + t.stages, stages.data(), sizeof(pa::StageTile) * stages.size());
+    if (!upload_tables(p)) {
+        cudaGetLastError();
+        if (fresh) pa_plan_destroy(p);
+        return PA_ERR_CUDA;
+    }
     *out = p;
     return PA_OK;
 }
@@ -302,7 +367,7 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     info->num_prefill_tiles = p->num_tiles;
     info->decode_kv_blocks = p->decode_blocks;
     info->prefill_causal_pairs = p->prefill_pairs;
-    info->table_bytes = p->ws.table_bytes;
+    info->table_bytes = p->tl.bytes;
     info->workspace_bytes = p->ws.total;
     info->num_staged_kv_tiles = p->num_stages;
     info->num_prefill_ctas = p->num_prefill_ctas;
@@ -313,8 +378,14 @@ extern "C" size_t pa_plan_workspace_bytes(const pa_plan *plan) { return plan ? p
 
 extern "C" void pa_plan_destroy(pa_plan *plan) {
     if (!plan) return;
-    wait_upload(plan);
+    {
+        DeviceScope scope(plan->device);
+        wait_idle(plan);
+        if (plan->d_tables) cudaFree(plan->d_tables);
+        if (plan->upload_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->upload_event));
+        if (plan->use_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->use_event));
+        if (plan->upload_stream) cudaStreamDestroy(static_cast<cudaStream_t>(plan->upload_stream));
+    }
     free_tables(plan);
-    if (plan->upload_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->upload_event));
     delete plan;
 }

@@ -36,19 +36,24 @@ struct DecodeRow {
 };
 
 // A decode warp's work: flat (row, block) range [start, next unit's start).
+// The first row's segment and key count are repeated here so that a warp
+// can start its first copies without first reading the row table.
 struct DecodeUnit {
     int32_t row;
     int32_t block;
+    int32_t seq;     // rows[row].seq (0 for the end marker)
+    int32_t n_keys;  // rows[row].n_keys (0 for the end marker)
 };
 
 // A row cut across several units.  Each unit writes its partial, then takes
-// a ticket from `arrived` (zero in the uploaded tables); the unit that takes
-// the last ticket merges the partials and writes the row.  Nobody waits.
+// a ticket from the row's counter (in the plan's device tables, zero after
+// every upload); the unit that takes the last ticket merges the partials,
+// writes the row and sets the counter back to zero.  Nobody waits.
 struct CombineRow {
     int32_t row;
     int32_t piece_base;
     int32_t piece_count;
-    int32_t arrived;
+    int32_t pad;
 };
 
 // One prefill work item: up to 128 consecutive queries of one segment for one
@@ -78,11 +83,18 @@ struct StageTile {
 
 constexpr size_t kStagedAlign = 1024;
 
+// The plan's tables, uploaded to a device buffer the plan owns: read-only
+// work lists, and one merge ticket counter per split row (zero between
+// calls: each call leaves them so).
+struct TableLayout {
+    size_t units = 0, rows = 0, combine = 0, tiles = 0, cta_start = 0, stages = 0, arrived = 0;  // byte offsets
+    size_t bytes = 0;
+};
+
+// The caller's workspace: the header (status word first) at offset 0, then
+// scratch that needs no initial value (split partials, staged K/V tiles).
 struct WorkspaceLayout {
-    // byte offsets; the header (status word first) is at offset 0
-    size_t header = 0, units = 0, rows = 0, combine = 0, tiles = 0, cta_start = 0, stages = 0;
-    size_t table_bytes = 0;                              // bytes copied from the plan
-    size_t partial_o = 0, partial_ml = 0, staged = 0;    // scratch offsets
+    size_t header = 0, partial_o = 0, partial_ml = 0, staged = 0;
     size_t total = 0;
 };
 
@@ -103,15 +115,22 @@ struct pa_plan {
     int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)
     int32_t num_stages = 0;              // staged K/V key tiles
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
+    pa::TableLayout tl;
     pa::WorkspaceLayout ws;
-    // Image of [header | units | rows | combine | tiles | cta_start | stages], copied into the workspace by
-    // every attention call.  Page-locked when a device is present, so that the
-    // copy is truly asynchronous; the event is recorded after each copy, and a
-    // rebuild or destroy waits on it before touching the buffer.
+    // Host image of the tables (page-locked when the plan has a device) and
+    // its device copy.  A build uploads the image on the plan's own stream
+    // and records upload_event; every attention call makes its stream wait
+    // for upload_event and records use_event after its last kernel.  A
+    // rebuild or destroy first waits for both, so that neither buffer
+    // changes under a queued copy or a running kernel.
     uint8_t *tables = nullptr;
     size_t tables_capacity = 0;
     bool tables_pinned = false;
-    void *upload_event = nullptr;        // cudaEvent_t, or null without a device
+    void *d_tables = nullptr;            // device buffer (cudaMalloc), d_capacity bytes
+    size_t d_capacity = 0;
+    void *upload_stream = nullptr;       // cudaStream_t (non-blocking), or null without a device
+    void *upload_event = nullptr;        // cudaEvent_t
+    void *use_event = nullptr;           // cudaEvent_t
     int device = -1;
 };
 

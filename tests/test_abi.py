@@ -82,7 +82,11 @@ def test_plan_invariants(lib, name):
     assert info["num_partials"] >= 2 * info["num_combine_rows"]
     assert info["num_partials"] <= info["num_combine_rows"] + info["num_decode_units"] * 2
     G = lay.num_q_heads // lay.num_kv_heads
-    assert info["workspace_bytes"] >= info["table_bytes"] + info["num_partials"] * G * lay.head_dim * 4
+    # the workspace holds the status word, one ticket per split row and the
+    # partials; the plan's own tables live in device memory the plan owns
+    assert info["table_bytes"] > 0
+    assert info["workspace_bytes"] >= 256 + info["num_partials"] * G * lay.head_dim * 4
+    assert info["table_bytes"] >= 4 * info["num_combine_rows"]
     assert plan.workspace_bytes == info["workspace_bytes"]
     # prefill tiles are dealt to at most one persistent CTA per SM; K/V of
     # every prefill segment are staged per kv head in 128-key tiles

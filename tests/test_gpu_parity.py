@@ -290,7 +290,7 @@ def test_traced_call_matches_and_times_each_kernel(cuda_lib):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
     t = tr.elapsed_ms()
-    assert t["decode"] > 0 and t["combine"] >= 0 and t["table_copy"] >= 0
+    assert t["decode"] > 0 and t["combine"] >= 0 and t["plan_wait"] >= 0
     tr2 = pa.Trace(stages=("decode",))
     pa.attention_varlen(b.q, kc, vc, bt, cu, sl, b.scale, out, plan, ws, trace=tr2)
     torch.cuda.synchronize()
