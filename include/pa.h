@@ -218,6 +218,10 @@ int pa_attention_varlen(const void *d_q, const void *d_k_cache, const void *d_v_
  *   [2] after the split-KV kernel      [3] = [2] (no separate combine kernel)
  *   [4] before the K/V staging and prefill kernels
  *   [5] after the prefill kernel
+ * When the plan runs the two kernels side by side (pa_plan_info
+ * num_prefill_ctas below the SM count while decode units exist), [1]-[3]
+ * are recorded on the side stream that runs the decode kernel and [4], [5]
+ * on `stream`, so both intervals measure their own kernel.
  * Events of stages that do not run are still recorded (adjacent), so every
  * interval is defined.  Results are identical to pa_attention_varlen.
  */

@@ -2,6 +2,7 @@
 // The declarations, with the meaning of every argument, are in include/pa.h.
 #include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -102,6 +103,26 @@ inline cudaError_t mark(const pa_trace *trace, int i, cudaStream_t stream) {
 }
 }  // namespace
 
+namespace {
+// Per-device stream of the least priority, created on first use, on which
+// the decode kernel runs when it shares the GPU with the prefill kernel.
+// Never destroyed (it lives as long as the process's context).
+cudaStream_t side_stream(int device) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    if (device < 0 || device >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[device]) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+        cudaStream_t s = nullptr;
+        if (cudaStreamCreateWithPriority(&s, cudaStreamNonBlocking, least) != cudaSuccess) return nullptr;
+        streams[device] = s;
+    }
+    return streams[device];
+}
+}  // namespace
+
 extern "C" int pa_attention_varlen(const void *q, const void *k_cache, const void *v_cache,
                                    const int32_t *block_tables, const int32_t *cu_seqlens_q,
                                    const int32_t *seq_lens, float scale, void *out,
@@ -147,9 +168,8 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
     if (cudaStreamWaitEvent(stream, static_cast<cudaEvent_t>(plan->upload_event), 0) != cudaSuccess)
         return PA_ERR_CUDA;
     const float scale_log2 = scale * kLog2e;
-    if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+    DecodeParams p{};
     if (plan->num_units > 0) {
-        DecodeParams p;
         p.q = static_cast<const __nv_bfloat16 *>(q);
         p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
         p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
@@ -168,14 +188,9 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.group = plan->group;
         p.max_blocks_per_seq = d.max_blocks_per_seq;
         p.scale_log2 = scale_log2;
-        if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 2, stream) != cudaSuccess) return PA_ERR_CUDA;
-    } else if (mark(trace, 2, stream) != cudaSuccess) {
-        return PA_ERR_CUDA;
     }
-    if (mark(trace, 3, stream) != cudaSuccess || mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
+    PrefillParams pp{};
     if (plan->num_tiles > 0) {
-        PrefillParams pp;
         pp.q = static_cast<const __nv_bfloat16 *>(q);
         pp.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
         pp.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
@@ -198,7 +213,41 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         pp.group = plan->group;
         pp.max_blocks_per_seq = d.max_blocks_per_seq;
         pp.scale_log2 = scale_log2;
+    }
+    const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
+    if (side_by_side) {
+        // The prefill kernel (persistent, one CTA per SM, on overlap_sms SMs)
+        // stays on the caller's stream, runnable as soon as the staging
+        // kernel ends, so that its CTAs are placed first; the decode kernel,
+        // sized for the other SMs, waits on a side stream of the least
+        // priority for the fork event and fills those SMs.
+        cudaStream_t side = side_stream(plan->device);
+        if (!side) return PA_ERR_CUDA;
+        cudaEvent_t fork = static_cast<cudaEvent_t>(plan->fork_event);
+        cudaEvent_t join = static_cast<cudaEvent_t>(plan->join_event);
+        if (mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (cudaEventRecord(fork, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (cudaStreamWaitEvent(side, fork, 0) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 1, side) != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_decode(p, d.head_dim, side) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 2, side) != cudaSuccess || mark(trace, 3, side) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;  // prefill, not the join
+        if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
+            return PA_ERR_CUDA;
+        if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+        return PA_OK;
+    } else {
+        if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess ||
+            mark(trace, 4, stream) != cudaSuccess)
+            return PA_ERR_CUDA;
+        if (plan->num_tiles > 0) {
+            if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+            if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        }
     }
     if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;
     // the plan's next build waits for this

@@ -62,6 +62,8 @@ struct PrefillParams {
     float scale_log2;
 };
 
+// Gathers the staged K/V tiles (must precede launch_prefill in stream order).
+cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream);
 
 // Data-dependent precondition checks; writes a nonzero flag word on failure.

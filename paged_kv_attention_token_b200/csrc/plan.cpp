@@ -44,6 +44,35 @@ constexpr int64_t kTileOverheadSteps = 2;
 // q, the final write or merge) stay small against the streaming.
 constexpr int64_t kMinBlocksPerUnit = 4;
 
+// Cost model for running the prefill kernel beside the decode kernel on
+// disjoint SMs (B200 measurements): one 128-key step of a two-head tile
+// takes a CTA (one SM) ~3.5 us; the decode kernel streams ~66 GB/s per SM
+// up to ~6.1 TB/s of HBM bandwidth (reached from ~92 SMs on).
+constexpr double kPrefillStepUs = 3.5;
+constexpr double kDecodeBytesPerUsPerSm = 66e3;
+constexpr double kHbmBytesPerUs = 6.1e6;
+constexpr int kMinSideSms = 8;  // fewest SMs either kernel is given when they share the GPU
+
+// SMs for the prefill kernel when it runs beside the decode kernel, or 0 when
+// running them one after the other is predicted to be as fast.
+int overlap_split(int num_sms, int64_t prefill_steps, int64_t decode_bytes) {
+    if (prefill_steps <= 0 || decode_bytes <= 0 || num_sms < 2 * kMinSideSms) return 0;
+    auto decode_us = [&](int sms) {
+        return (double)decode_bytes / std::min(kHbmBytesPerUs, sms * kDecodeBytesPerUsPerSm);
+    };
+    const double serial = prefill_steps * kPrefillStepUs / num_sms + decode_us(num_sms);
+    double best = serial;
+    int best_p = 0;
+    for (int s = kMinSideSms; s <= num_sms - kMinSideSms; ++s) {
+        const double t = std::max(prefill_steps * kPrefillStepUs / s, decode_us(num_sms - s));
+        if (t < best) {
+            best = t;
+            best_p = s;
+        }
+    }
+    return best_p;
+}
+
 // Scoped switch to the plan's device (plans own device memory, a stream and
 // events, which belong to the device they were made on).
 struct DeviceScope {
@@ -115,7 +144,7 @@ bool create_sync_objects(pa_plan *p) {
         if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
         p->upload_stream = s;
     }
-    for (void **slot : {&p->upload_event, &p->use_event}) {
+    for (void **slot : {&p->upload_event, &p->use_event, &p->fork_event, &p->join_event}) {
         if (*slot) continue;
         cudaEvent_t e = nullptr;
         if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
@@ -231,7 +260,17 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
                          return a.n_kv_tiles > b.n_kv_tiles;
                      });
     // Deal the tiles to persistent CTAs; each CTA's tiles become contiguous.
-    const int grid = (int)std::min<size_t>(tiles.size(), (size_t)p->num_sms);
+    // Decode KV bytes and prefill steps decide whether the two kernels share
+    // the GPU side by side, and on how many SMs each runs.
+    int64_t decode_blocks_all = 0;
+    for (const pa::DecodeRow &r : rows) decode_blocks_all += cdiv(r.n_keys, pa::kBlockSize);
+    int64_t prefill_steps = 0;
+    for (const pa::PrefillTile &t : tiles) prefill_steps += t.n_kv_tiles + kTileOverheadSteps;
+    p->overlap_sms = overlap_split(p->num_sms, prefill_steps,
+                                   decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2);
+    const int prefill_sms = p->overlap_sms > 0 ? p->overlap_sms : p->num_sms;
+    const int decode_sms = p->num_sms - p->overlap_sms;
+    const int grid = (int)std::min<size_t>(tiles.size(), (size_t)prefill_sms);
     std::vector<int32_t> cta_start(grid + 1, 0);
     if (grid > 0) {
         std::vector<std::vector<int32_t>> per(grid);
@@ -262,7 +301,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     const int64_t total = prefix[R];
     int64_t P = 0;
     if (total > 0) {
-        const int64_t max_units = (int64_t)p->num_sms * pa::decode_units_per_sm(d.head_dim);
+        const int64_t max_units = (int64_t)decode_sms * pa::decode_units_per_sm(d.head_dim);
         P = std::max<int64_t>(1, std::min(max_units, cdiv(total, kMinBlocksPerUnit)));
     }
     std::vector<pa::DecodeUnit> units(P + 1);
@@ -383,7 +422,8 @@ extern "C" void pa_plan_destroy(pa_plan *plan) {
         wait_idle(plan);
         if (plan->d_tables) cudaFree(plan->d_tables);
         if (plan->upload_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->upload_event));
-        if (plan->use_event) cudaEventDestroy(static_cast<cudaEvent_t>(plan->use_event));
+        for (void *e : {plan->use_event, plan->fork_event, plan->join_event})
+            if (e) cudaEventDestroy(static_cast<cudaEvent_t>(e));
         if (plan->upload_stream) cudaStreamDestroy(static_cast<cudaStream_t>(plan->upload_stream));
     }
     free_tables(plan);

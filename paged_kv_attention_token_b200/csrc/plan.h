@@ -113,6 +113,7 @@ struct pa_plan {
     // prefill part
     int32_t num_tiles = 0;
     int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)
+    int32_t overlap_sms = 0;             // > 0: prefill runs on this many SMs beside the decode kernel
     int32_t num_stages = 0;              // staged K/V key tiles
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::TableLayout tl;
@@ -131,6 +132,8 @@ struct pa_plan {
     void *upload_stream = nullptr;       // cudaStream_t (non-blocking), or null without a device
     void *upload_event = nullptr;        // cudaEvent_t
     void *use_event = nullptr;           // cudaEvent_t
+    void *fork_event = nullptr;          // cudaEvent_t: decode and prefill run side by side
+    void *join_event = nullptr;          // cudaEvent_t
     int device = -1;
 };
 

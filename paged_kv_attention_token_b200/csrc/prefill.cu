@@ -632,7 +632,6 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    stage_kernel<D><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
     prefill_kernel<D><<<p.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(p, maps);
     return cudaGetLastError();
 }
@@ -640,6 +639,15 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
 }  // namespace
 
 bool prefill_kernel_available() { return true; }
+
+cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stream) {
+    if (p.num_stages == 0) return cudaSuccess;
+    if (head_dim == 64)
+        stage_kernel<64><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
+    else
+        stage_kernel<128><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream) {
     if (p.num_tiles == 0) return cudaSuccess;
