@@ -46,9 +46,10 @@ constexpr int64_t kMinBlocksPerUnit = 4;
 
 // Cost model for running the prefill kernel beside the decode kernel on
 // disjoint SMs (B200 measurements): one 128-key step of a two-head tile
-// takes a CTA (one SM) ~3.5 us; the decode kernel streams ~66 GB/s per SM
+// takes a CTA (one SM) ~2.9 us when the prefill kernel has a part of the
+// GPU (~3.5 us with all SMs); the decode kernel streams ~66 GB/s per SM
 // up to ~6.1 TB/s of HBM bandwidth (reached from ~92 SMs on).
-constexpr double kPrefillStepUs = 3.5;
+constexpr double kPrefillStepUs = 2.9;
 constexpr double kDecodeBytesPerUsPerSm = 66e3;
 constexpr double kHbmBytesPerUs = 6.1e6;
 constexpr int kMinSideSms = 8;  // fewest SMs either kernel is given when they share the GPU
