@@ -72,25 +72,18 @@ def step_bytes(lay: W.Layout) -> dict:
     return {"kv": kv, "qo": qo, "scatter": scatter, "meta": meta, "total": kv + qo + scatter + meta}
 
 
-def decode_prefill_split(lay: W.Layout):
-    """Algorithmic work of the two kernels: the decode kernel's distinct KV
-    bytes (+ q/out of its rows) and the prefill kernel's flops (4 D per
-    causal (query, key) pair and query head) and bytes."""
-    Hq, Hkv, D = lay.num_q_heads, lay.num_kv_heads, lay.head_dim
-    per_tok = 2 * Hkv * D * 2
+def decode_prefill_split(lay: W.Layout, info: dict):
+    """Algorithmic work of the two kernels, from the plan: the decode
+    kernel's KV bytes (the blocks its rows read: all of a row's keys, or
+    those after a shared prefix the prefill kernel attends) + q/out of its
+    rows, and the prefill kernel's flops (4 D per (query, visible key) pair
+    and query head, shared-prefix pairs included) and q/out bytes."""
+    Hq, D = lay.num_q_heads, lay.head_dim
     dec = lay.q_lens <= 16
     dec_tokens = int(lay.q_lens[dec].sum())
-    if lay.shared_prefix_blocks and dec.all():
-        kv_dec = lay.kv_bytes_read()
-    else:
-        kv_dec = per_tok * int(lay.seq_lens[dec].astype(np.int64).sum())
-    pairs = 0
-    for L, n in zip(lay.q_lens[~dec].astype(np.int64), lay.seq_lens[~dec].astype(np.int64)):
-        pairs += int(L * (n - L) + L * (L + 1) // 2)
-    flops = 4 * D * Hq * pairs
-    kv_pre = per_tok * int(lay.seq_lens[~dec].astype(np.int64).sum())
-    return {"decode_bytes": kv_dec + 2 * dec_tokens * Hq * D * 2, "prefill_flops": flops,
-            "prefill_bytes": kv_pre + 2 * int(lay.q_lens[~dec].sum()) * Hq * D * 2}
+    kv_dec = int(info["decode_kv_blocks"]) * 16 * D * 2 * 2
+    flops = 4 * D * Hq * int(info["prefill_causal_pairs"])
+    return {"decode_bytes": kv_dec + 2 * dec_tokens * Hq * D * 2, "prefill_flops": flops}
 
 
 def is_decode_workload(lay: W.Layout) -> bool:
@@ -326,10 +319,11 @@ def run_ours(args):
     acct = step_bytes(lay)
     bt, cu, sl, slots = batch.device_ints(dev)
     h_cu, h_sl = lay.cu_seqlens_q, lay.seq_lens
+    h_bt = lay.block_tables  # host copy: lets the planner find shared prefixes
     kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
     out = torch.empty_like(batch.q)
     dims = dims_for(pa, lay)
-    plan0 = pa.Plan(h_cu, h_sl, dims, device=local)
+    plan0 = pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt)
     info = plan0.info()
     ws = pa.workspace_for(plan0, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -338,13 +332,13 @@ def run_ours(args):
     launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + (1 if info["num_prefill_tiles"] else 0)
 
     # two plans rebuilt in turn, as an engine keeps them across steps
-    plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local), pa.Plan(h_cu, h_sl, dims, device=local)]
+    plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt), pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt)]
     step_no = [0]
 
     def one_step(trace=None, ev=None):
         flush.fill_(1)
         t0 = time.perf_counter()
-        plan = plan_pool[step_no[0] % 2].rebuild(h_cu, h_sl, dims)
+        plan = plan_pool[step_no[0] % 2].rebuild(h_cu, h_sl, dims, h_bt)
         step_no[0] += 1
         plan_s = time.perf_counter() - t0
         if ev is not None:
@@ -411,7 +405,7 @@ def run_ours(args):
     comb_ms = statistics.mean(s["combine"] for s in other)
     wait_ms = statistics.mean(s["plan_wait"] for s in other)
     prefill_ms = statistics.mean(s["prefill"] for s in other)
-    split = decode_prefill_split(lay)
+    split = decode_prefill_split(lay, info)
     roofline_decode = roofline_prefill = None
     dec_bytes = split["decode_bytes"]
     if dec_bytes and dec_ms > 0:
@@ -472,7 +466,7 @@ def run_ours(args):
             e0.record(stream)
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
-            plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims)
+            plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims, h_bt)
             pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)
             pa.attention_varlen(dev_in["q"], kc, vc, dev_in["bt"], dev_in["cu"], dev_in["sl"],
                                 batch.scale, out, plan, ws, stream=stream)

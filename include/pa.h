@@ -112,6 +112,18 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  * GPU work a build queues).
  *   h_cu_seqlens_q  host [S+1] int32
  *   h_seq_lens      host [S] int32
+ *   h_block_tables  host [S][MB] int32 (the values the device array will
+ *                   hold), or NULL.  Given, the planner looks for shared
+ *                   prefixes ("vLLM 学习笔记 01" §2.2, prefix caching: requests
+ *                   whose tables start with the same physical blocks): runs
+ *                   of at least 4 consecutive single-token segments whose
+ *                   first 16 or more table entries agree.  For such a run the
+ *                   prefill kernel attends all its tokens to the shared
+ *                   blocks at once (a dense tensor-core pass that reads them
+ *                   once per kv head) and leaves partials, and the decode
+ *                   kernel reads only each row's later blocks and merges.
+ *                   Only the first ceil(seq_len / 16) entries of a row are
+ *                   read.
  *   dims            host; T, S, Hq, Hkv, D, B are used
  *   device          CUDA device ordinal the plan is built for (its SM count
  *                   is read once per process and cached; the device tables
@@ -140,7 +152,8 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  */
 typedef struct pa_plan pa_plan;
 int pa_plan_build(const int32_t *h_cu_seqlens_q, const int32_t *h_seq_lens,
-                  const pa_dims *dims, int device, pa_plan **out);
+                  const int32_t *h_block_tables, const pa_dims *dims, int device,
+                  pa_plan **out);
 
 /* What a plan holds, for tests, logging and roofline accounting. */
 typedef struct {
@@ -157,6 +170,8 @@ typedef struct {
     int32_t num_staged_kv_tiles;  /* 128-key K/V tiles of prefill segments gathered
                                      into the workspace (per kv head) */
     int32_t num_prefill_ctas;     /* persistent CTAs of the prefill kernel */
+    int32_t num_prefix_groups;    /* shared-prefix runs found (h_block_tables given) */
+    int32_t reserved;
 } pa_plan_info;
 int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
 

@@ -65,7 +65,8 @@ class PlanInfo(ctypes.Structure):
                 ("num_combine_rows", ctypes.c_int32), ("num_prefill_tiles", ctypes.c_int32),
                 ("decode_kv_blocks", ctypes.c_int64), ("prefill_causal_pairs", ctypes.c_int64),
                 ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
-                ("num_staged_kv_tiles", ctypes.c_int32), ("num_prefill_ctas", ctypes.c_int32)]
+                ("num_staged_kv_tiles", ctypes.c_int32), ("num_prefill_ctas", ctypes.c_int32),
+                ("num_prefix_groups", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     def as_dict(self):
         return {n: int(getattr(self, n)) for n, _ in self._fields_}
@@ -85,7 +86,7 @@ def load_library():
         DP = ctypes.POINTER(Dims)
         sig = {
             "pa_reshape_and_cache": (I, [P, P, P, P, P, DP, P]),
-            "pa_plan_build": (I, [P, P, DP, I, ctypes.POINTER(P)]),
+            "pa_plan_build": (I, [P, P, P, DP, I, ctypes.POINTER(P)]),
             "pa_plan_get_info": (I, [P, ctypes.POINTER(PlanInfo)]),
             "pa_plan_workspace_bytes": (SZ, [P]),
             "pa_plan_destroy": (None, [P]),
@@ -180,23 +181,30 @@ class Plan:
 
     The plan must stay alive until the GPU work queued with it has completed
     (like every other input).  ``rebuild`` re-partitions for the next step in
-    place, reusing the plan's page-locked buffer."""
+    place, reusing the plan's buffers.  With host ``block_tables`` ([S][MB]
+    int32, the values of the device array), runs of decodes that share
+    their leading blocks are attended to them once (cascade)."""
 
-    def __init__(self, cu_seqlens_q, seq_lens, dims: Dims, device: int | None = None):
+    def __init__(self, cu_seqlens_q, seq_lens, dims: Dims, device: int | None = None, block_tables=None):
         lib = load_library()
         self._lib = lib
         if device is None:
             device = torch.cuda.current_device() if torch.cuda.is_available() else -1
         self.device = int(device)
         self._h = ctypes.c_void_p()
-        self.rebuild(cu_seqlens_q, seq_lens, dims)
+        self.rebuild(cu_seqlens_q, seq_lens, dims, block_tables)
 
-    def rebuild(self, cu_seqlens_q, seq_lens, dims: Dims):
+    def rebuild(self, cu_seqlens_q, seq_lens, dims: Dims, block_tables=None):
         self._cu = _host_i32(cu_seqlens_q, "cu_seqlens_q")
         self._sl = _host_i32(seq_lens, "seq_lens")
+        self._bt = None if block_tables is None else _host_i32(block_tables, "block_tables")
         self.dims = Dims(*[getattr(dims, n) for n, _ in Dims._fields_])
+        if self._bt is not None and (self._bt.ndim != 2 or self._bt.shape[0] != self.dims.num_seqs
+                                     or self._bt.shape[1] != self.dims.max_blocks_per_seq):
+            raise ValueError(f"block_tables must be [{self.dims.num_seqs}][{self.dims.max_blocks_per_seq}]")
+        bt_ptr = None if self._bt is None else self._bt.ctypes.data_as(ctypes.c_void_p)
         _check(self._lib.pa_plan_build(self._cu.ctypes.data_as(ctypes.c_void_p),
-                                       self._sl.ctypes.data_as(ctypes.c_void_p),
+                                       self._sl.ctypes.data_as(ctypes.c_void_p), bt_ptr,
                                        ctypes.byref(self.dims), self.device, ctypes.byref(self._h)),
                "pa_plan_build")
         return self

@@ -204,6 +204,10 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         pp.stages = reinterpret_cast<const StageTile *>(tb + tl.stages);
         pp.staged = ws + w.staged;
         pp.num_stages = plan->num_stages;
+        pp.rows = reinterpret_cast<const DecodeRow *>(tb + tl.rows);
+        pp.combine = reinterpret_cast<const CombineRow *>(tb + tl.combine);
+        pp.partial_o = reinterpret_cast<float *>(ws + w.partial_o);
+        pp.partial_ml = reinterpret_cast<float2 *>(ws + w.partial_ml);
         pp.status = reinterpret_cast<uint32_t *>(ws + w.header);
         pp.num_tiles = plan->num_tiles;
         pp.num_tokens = d.num_tokens;
@@ -236,6 +240,16 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;  // prefill, not the join
         if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
             return PA_ERR_CUDA;
+        if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+        return PA_OK;
+    } else if (plan->cascade) {
+        // shared-prefix partials first; the decode kernel merges them
+        if (mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 5, stream) != cudaSuccess || mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
         return PA_OK;
     } else {

@@ -313,13 +313,21 @@ __device__ __forceinline__ void cursor_set_row(const DecodeParams &p, const Deco
     c.bt_base = -1;
 }
 
+// Moves the cursor to the start of row c.r (its first_block), or marks it
+// done when the warp's run ends before that.
 __device__ __forceinline__ void cursor_enter_row(const DecodeParams &p, const DecodeUnit &end,
                                                  LoadCursor &c) {
+    // (the run end of the last unit is row R, block 0: never read)
     if (c.r > end.row || (c.r == end.row && end.block == 0)) {
         c.done = true;
         return;
     }
     const DecodeRow row = p.rows[c.r];
+    if (c.r == end.row && end.block <= row.first_block) {
+        c.done = true;
+        return;
+    }
+    c.b = row.first_block;
     cursor_set_row(p, end, c, row.seq, row.n_keys);
 }
 
@@ -372,25 +380,25 @@ __device__ __forceinline__ void issue_step(const DecodeParams &p, const DecodeUn
     }
     c.b += NB;
     if (c.b >= c.bend) {
-        c.b = 0;
         ++c.r;
         cursor_enter_row(p, end, c);
     }
 }
 
-// Walks a warp's run piece by piece: fn(row_index, row, b0, bend).
+// Walks a warp's run piece by piece: fn(row_index, row, b0, bend), blocks
+// [b0, bend) of the row's block table (a row's range starts at its
+// first_block; the run may start inside its first row).
 template <typename F>
 __device__ __forceinline__ void for_each_piece(const DecodeParams &p, int unit, F &&fn) {
     const DecodeUnit start = p.units[unit];
     const DecodeUnit end = p.units[unit + 1];
-    int r = start.row, b0 = start.block;
-    while (r < end.row || (r == end.row && b0 < end.block)) {
+    for (int r = start.row; r <= end.row; ++r) {
+        if (r == end.row && end.block == 0) break;  // (row R of the last unit's end is never read)
         const DecodeRow row = p.rows[r];
-        const int nblk = (row.n_keys + 15) >> 4;
-        const int bend = (r == end.row) ? end.block : nblk;
+        const int b0 = r == start.row ? start.block : row.first_block;
+        const int bend = r == end.row ? end.block : (row.n_keys + 15) >> 4;
+        if (b0 >= bend) break;
         fn(r, row, b0, bend);
-        ++r;
-        b0 = 0;
     }
 }
 
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
             __syncwarp();
             int last = 0;
             const CombineRow c = p.combine[row.combine];
-            if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.piece_count - 1;
+            if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.tickets - 1;
             last = __shfl_sync(kFullMask, last, 0);
             if (last) {
                 __threadfence();

@@ -49,6 +49,11 @@ struct PrefillParams {
     const int32_t *cta_start;  // CTA c owns tiles [cta_start[c], cta_start[c + 1])
     const StageTile *stages;   // the gather kernel's list
     uint8_t *staged;          // staged K/V tiles (workspace)
+    // shared-prefix tiles write partials of the decode rows they serve
+    const DecodeRow *rows;
+    const CombineRow *combine;
+    float *partial_o;         // [pieces][G][D]
+    float2 *partial_ml;       // [pieces][G]: (max in log2 units, sum)
     uint32_t *status;
     int num_tiles;
     int num_ctas;

@@ -54,6 +54,54 @@ constexpr double kDecodeBytesPerUsPerSm = 66e3;
 constexpr double kHbmBytesPerUs = 6.1e6;
 constexpr int kMinSideSms = 8;  // fewest SMs either kernel is given when they share the GPU
 
+// Shared-prefix (cascade) groups: runs of at least kMinGroupSegs consecutive
+// single-token segments whose first kMinSharedBlocks or more block-table
+// entries are the same physical blocks.
+constexpr int kMinGroupSegs = 4;
+constexpr int kMinSharedBlocks = 16;
+
+struct PrefixGroup {
+    int seg0, nseg;  // segments seg0 .. seg0 + nseg - 1
+    int blocks;      // shared leading blocks
+};
+
+// Groups of consecutive single-token segments that share their leading
+// blocks; each query sits past the shared keys, so all of them see all of
+// them.
+std::vector<PrefixGroup> find_prefix_groups(const int32_t *h_cu, const int32_t *h_seq, const int32_t *h_bt,
+                                            const pa_dims &d) {
+    std::vector<PrefixGroup> groups;
+    if (!h_bt) return groups;
+    const int S = d.num_seqs, MB = d.max_blocks_per_seq;
+    auto single = [&](int i) { return h_cu[i + 1] - h_cu[i] == 1; };
+    int i = 0;
+    while (i < S) {
+        if (!single(i) || h_seq[i] < 2) {
+            ++i;
+            continue;
+        }
+        const int32_t *bi = h_bt + (size_t)i * MB;
+        int c = (h_seq[i] - 1) / pa::kBlockSize;  // blocks wholly before the query's own key
+        int j = i + 1;
+        while (j < S && single(j) && h_seq[j] >= 2) {
+            const int32_t *bj = h_bt + (size_t)j * MB;
+            const int cap = std::min(c, (h_seq[j] - 1) / pa::kBlockSize);
+            int k = 0;
+            while (k < cap && bj[k] == bi[k]) ++k;
+            if (k < kMinSharedBlocks) break;
+            c = k;
+            ++j;
+        }
+        if (j - i >= kMinGroupSegs && c >= kMinSharedBlocks) {
+            groups.push_back({i, j - i, c});
+            i = j;
+        } else {
+            ++i;
+        }
+    }
+    return groups;
+}
+
 // SMs for the prefill kernel when it runs beside the decode kernel, or 0 when
 // running them one after the other is predicted to be as fast.
 int overlap_split(int num_sms, int64_t prefill_steps, int64_t decode_bytes) {
@@ -192,8 +240,8 @@ int check_dims(const pa_dims *d) {
 
 }  // namespace
 
-extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa_dims *dims,
-                             int device, pa_plan **out) {
+extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const int32_t *h_bt,
+                             const pa_dims *dims, int device, pa_plan **out) {
     if (!out) return PA_ERR_NULL;
     int st = check_dims(dims);
     if (st != PA_OK) return st;
@@ -229,32 +277,74 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     p->prefill_pairs = 0;
     const int Hkv = d.num_kv_heads;
 
+    const int G = d.num_q_heads / d.num_kv_heads;
     std::vector<pa::DecodeRow> rows;
     std::vector<pa::PrefillTile> tiles;
     std::vector<pa::StageTile> stages;
+    // shared prefixes: the prefill kernel attends each group's tokens to the
+    // shared blocks (key splits of them, as partials); the decode rows read
+    // only the blocks after them
+    const std::vector<PrefixGroup> groups =
+        pa::prefill_kernel_available() ? find_prefix_groups(h_cu, h_seq, h_bt, d) : std::vector<PrefixGroup>();
+    std::vector<int> shared(d.num_seqs, 0), group_of(d.num_seqs, -1), seg_row0(d.num_seqs, -1);
+    for (size_t k = 0; k < groups.size(); ++k)
+        for (int i = groups[k].seg0; i < groups[k].seg0 + groups[k].nseg; ++i) {
+            shared[i] = groups[k].blocks;
+            group_of[i] = (int)k;
+        }
+    std::vector<int> group_splits(groups.size(), 0);
     for (int i = 0; i < d.num_seqs; ++i) {
         const int L = h_cu[i + 1] - h_cu[i];
         const int n = h_seq[i];
         if (L == 0) continue;
         if (L <= pa::kDecodeMaxQLen || !pa::prefill_kernel_available()) {
+            seg_row0[i] = (int)rows.size();
             for (int j = 0; j < L; ++j)
                 for (int g = 0; g < Hkv; ++g)
-                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, {0, 0, 0}});
+                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, shared[i], {0, 0}});
         } else {
-            const int G = d.num_q_heads / d.num_kv_heads;
             const int nt = (int)cdiv(n, pa::kPrefillTileN);  // key tiles of the segment
             const int base = (int)stages.size();
             for (int g = 0; g < Hkv; ++g)
-                for (int j = 0; j < nt; ++j) stages.push_back({i, g, j, 0});
+                for (int j = 0; j < nt; ++j) stages.push_back({i, g, j, n});
             for (int q0 = 0; q0 < L; q0 += pa::kPrefillTileM) {
                 const int last = std::min(L, q0 + pa::kPrefillTileM) - 1;
                 const int kv_tiles = (int)cdiv(n - L + last + 1, pa::kPrefillTileN);
                 for (int g = 0; g < Hkv; ++g)
                     for (int h = g * G; h < (g + 1) * G; h += 2)
-                        tiles.push_back({i, q0, h, kv_tiles, std::min(2, (g + 1) * G - h), base + g * nt, {0, 0}});
+                        tiles.push_back({i, q0, h, kv_tiles, std::min(2, (g + 1) * G - h), base + g * nt, 0, 0,
+                                         -1, 0, 0, 0});
             }
             for (int j = 0; j < L; ++j) p->prefill_pairs += n - L + j + 1;
         }
+    }
+    // Shared-prefix tiles: per group, chunk of up to 128 tokens, kv head,
+    // query-head pair and key split.  The key splits make enough tiles to
+    // fill the GPU without cutting a split below four 128-key tiles.
+    for (size_t k = 0; k < groups.size(); ++k) {
+        const PrefixGroup &gr = groups[k];
+        const int keys = gr.blocks * pa::kBlockSize;
+        const int nt = (int)cdiv(keys, pa::kPrefillTileN);
+        const int chunks = (int)cdiv(gr.nseg, pa::kPrefillTileM);
+        const int base_tiles = chunks * Hkv * (int)cdiv(G, 2);
+        const int splits = (int)std::max<int64_t>(
+            1, std::min<int64_t>(cdiv(nt, 4), cdiv(2 * (int64_t)p->num_sms, base_tiles)));
+        group_splits[k] = splits;
+        const int base = (int)stages.size();
+        for (int g = 0; g < Hkv; ++g)
+            for (int j = 0; j < nt; ++j) stages.push_back({gr.seg0, g, j, keys});
+        for (int c = 0; c < chunks; ++c) {
+            const int s0 = gr.seg0 + c * pa::kPrefillTileM;
+            const int q_rows = std::min(pa::kPrefillTileM, gr.seg0 + gr.nseg - s0);
+            for (int g = 0; g < Hkv; ++g)
+                for (int h = g * G; h < (g + 1) * G; h += 2)
+                    for (int sp = 0; sp < splits; ++sp) {
+                        const int t0 = (int)((int64_t)nt * sp / splits), t1 = (int)((int64_t)nt * (sp + 1) / splits);
+                        tiles.push_back({gr.seg0, h_cu[s0], h, t1 - t0, std::min(2, (g + 1) * G - h), base + g * nt,
+                                         t0, keys, seg_row0[s0] + g, sp, q_rows, 0});
+                    }
+        }
+        p->prefill_pairs += (int64_t)gr.nseg * keys;
     }
     std::stable_sort(tiles.begin(), tiles.end(),
                      [](const pa::PrefillTile &a, const pa::PrefillTile &b) {
@@ -264,10 +354,14 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     // Decode KV bytes and prefill steps decide whether the two kernels share
     // the GPU side by side, and on how many SMs each runs.
     int64_t decode_blocks_all = 0;
-    for (const pa::DecodeRow &r : rows) decode_blocks_all += cdiv(r.n_keys, pa::kBlockSize);
+    for (const pa::DecodeRow &r : rows) decode_blocks_all += cdiv(r.n_keys, pa::kBlockSize) - r.first_block;
     int64_t prefill_steps = 0;
     for (const pa::PrefillTile &t : tiles) prefill_steps += t.n_kv_tiles + kTileOverheadSteps;
-    p->overlap_sms = overlap_split(p->num_sms, prefill_steps,
+    // the decode kernel merges shared-prefix partials, so it follows the
+    // prefill kernel when there are any
+    p->cascade = !groups.empty();
+    p->num_prefix_groups = (int32_t)groups.size();
+    p->overlap_sms = p->cascade ? 0 : overlap_split(p->num_sms, prefill_steps,
                                    decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2);
     const int prefill_sms = p->overlap_sms > 0 ? p->overlap_sms : p->num_sms;
     const int decode_sms = p->num_sms - p->overlap_sms;
@@ -298,7 +392,8 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
     // Cut the decode rows' blocks into equal runs.
     const int64_t R = (int64_t)rows.size();
     std::vector<int64_t> prefix(R + 1, 0);
-    for (int64_t r = 0; r < R; ++r) prefix[r + 1] = prefix[r] + cdiv(rows[r].n_keys, pa::kBlockSize);
+    for (int64_t r = 0; r < R; ++r)
+        prefix[r + 1] = prefix[r] + cdiv(rows[r].n_keys, pa::kBlockSize) - rows[r].first_block;
     const int64_t total = prefix[R];
     int64_t P = 0;
     if (total > 0) {
@@ -313,8 +408,8 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
             const int64_t f = P ? total * u / P : 0;
             ustart[u] = f;
             while (r < R && prefix[r + 1] <= f) ++r;  // row holding block f
-            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)]), r < R ? rows[r].seq : 0,
-                        r < R ? rows[r].n_keys : 0};
+            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)]) + (r < R ? rows[r].first_block : 0),
+                        r < R ? rows[r].seq : 0, r < R ? rows[r].n_keys : 0};
         }
         units[P] = {(int32_t)R, 0, 0, 0};
     }
@@ -328,11 +423,15 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const pa
             int64_t v = u;
             while (v + 1 < P && ustart[v + 1] <= prefix[r + 1] - 1) ++v;  // unit of the last block
             const int32_t count = (int32_t)(v - u + 1);
-            if (count > 1) {
-                rows[r].slot_base = piece_base - (int32_t)u;
+            // partials of the row's shared prefix (written by the prefill
+            // kernel) come first
+            const int sg = group_of[rows[r].seq];
+            const int32_t pre = sg >= 0 ? group_splits[sg] : 0;
+            if (count > 1 || pre > 0) {
+                rows[r].slot_base = piece_base + pre - (int32_t)u;
                 rows[r].combine = (int32_t)combine.size();
-                combine.push_back({(int32_t)r, piece_base, count, 0});
-                piece_base += count;
+                combine.push_back({(int32_t)r, piece_base, count + pre, count});
+                piece_base += count + pre;
             }
         }
     }
@@ -411,6 +510,8 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     info->workspace_bytes = p->ws.total;
     info->num_staged_kv_tiles = p->num_stages;
     info->num_prefill_ctas = p->num_prefill_ctas;
+    info->num_prefix_groups = p->num_prefix_groups;
+    info->reserved = 0;
     return PA_OK;
 }
 

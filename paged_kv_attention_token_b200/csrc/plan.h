@@ -26,16 +26,20 @@ constexpr int32_t kUnsplitRow = INT32_MIN;
 // One decode row: a query token and one kv head (the G query heads of that
 // kv head are computed together).  Row id r = token_row * Hkv + kv_head.
 struct DecodeRow {
-    int32_t token;      // flat token index t
-    int32_t seq;        // segment index i (block-table row)
-    int32_t n_keys;     // keys this query sees: p + 1
-    int32_t slot_base;  // kUnsplitRow: one warp covers the row and writes out
-                        // directly; else partial slot of unit u is slot_base + u
-    int32_t combine;    // index of the row's CombineRow (split rows only)
-    int32_t pad[3];
+    int32_t token;        // flat token index t
+    int32_t seq;          // segment index i (block-table row)
+    int32_t n_keys;       // keys this query sees: p + 1
+    int32_t slot_base;    // kUnsplitRow: one warp covers the row and writes out
+                          // directly; else partial slot of unit u is slot_base + u
+    int32_t combine;      // index of the row's CombineRow (split rows only)
+    int32_t first_block;  // first block read here: > 0 when the row's leading
+                          // blocks are a prefix shared with other rows,
+                          // attended by the prefill kernel (cascade)
+    int32_t pad[2];
 };
 
-// A decode warp's work: flat (row, block) range [start, next unit's start).
+// A decode warp's work: flat (row, block) range [start, next unit's start);
+// blocks are block-table indices (a row's range starts at its first_block).
 // The first row's segment and key count are repeated here so that a warp
 // can start its first copies without first reading the row table.
 struct DecodeUnit {
@@ -45,27 +49,38 @@ struct DecodeUnit {
     int32_t n_keys;  // rows[row].n_keys (0 for the end marker)
 };
 
-// A row cut across several units.  Each unit writes its partial, then takes
-// a ticket from the row's counter (in the plan's device tables, zero after
-// every upload); the unit that takes the last ticket merges the partials,
-// writes the row and sets the counter back to zero.  Nobody waits.
+// A row whose result is merged from partials: cut across several decode
+// units, and/or with a shared prefix attended by the prefill kernel (whose
+// partials come first, written before the decode kernel starts).  Each
+// decode unit writes its partial, then takes a ticket from the row's counter
+// (in the plan's device tables, zero after every upload); the unit that
+// takes the last ticket merges all pieces, writes the row and sets the
+// counter back to zero.  Nobody waits.
 struct CombineRow {
     int32_t row;
     int32_t piece_base;
-    int32_t piece_count;
-    int32_t pad;
+    int32_t piece_count;  // all partials: prefix pieces, then the decode units'
+    int32_t tickets;      // decode units covering the row
 };
 
 // One prefill work item: up to 128 consecutive queries of one segment for one
 // or two query heads that share a kv head.
 struct PrefillTile {
-    int32_t seq;        // segment index
-    int32_t q_start;    // first query of the tile within the segment (j)
+    int32_t seq;        // segment index (its block table holds the keys)
+    int32_t q_start;    // first query: within the segment (j), or for a
+                        // shared-prefix tile the flat token index
     int32_t head;       // first query head
     int32_t n_kv_tiles; // 128-key tiles the tile reads
     int32_t num_heads;  // 1 or 2 (head and head + 1)
     int32_t kv_base;    // staged tile index of key tile 0 of (seq, kv head)
-    int32_t pad[2];
+    int32_t kv_tile0;   // first key tile read (a key split of a shared prefix)
+    int32_t key_limit;  // shared-prefix tile: every query sees keys < key_limit
+    int32_t row_base;   // shared-prefix tile: decode row of its first token for
+                        // this kv head (row of token k: row_base + k * Hkv);
+                        // -1 for a causal tile of a prefill segment
+    int32_t piece;      // shared-prefix tile: its piece among the row's partials
+    int32_t q_rows;     // shared-prefix tile: query tokens (consecutive)
+    int32_t pad;
 };
 
 // One staged key tile: keys 128 j .. 128 j + 127 of segment `seq` for one kv
@@ -77,8 +92,9 @@ struct PrefillTile {
 struct StageTile {
     int32_t seq;
     int32_t kv_head;
-    int32_t tile;  // j
-    int32_t pad;
+    int32_t tile;    // j
+    int32_t n_keys;  // keys that exist (the segment's length, or a shared
+                     // prefix's): rows of the tile at or past it are zeroed
 };
 
 constexpr size_t kStagedAlign = 1024;
@@ -114,6 +130,8 @@ struct pa_plan {
     int32_t num_tiles = 0;
     int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)
     int32_t overlap_sms = 0;             // > 0: prefill runs on this many SMs beside the decode kernel
+    bool cascade = false;                // shared-prefix tiles: the prefill kernel runs first
+    int32_t num_prefix_groups = 0;
     int32_t num_stages = 0;              // staged K/V key tiles
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::TableLayout tl;

@@ -223,16 +223,17 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk
 // TMEM, releases O (o_free) for the next tile's first PV, then divides by
 // its sum and writes bf16.
 template <int D>
-__device__ __forceinline__ void softmax_tile(const PrefillParams &p, uint32_t trow, uint32_t s_col, uint32_t o_col,
-                                             uint64_t *s_full, uint64_t *p_full, uint64_t *o_done, uint64_t *o_free,
-                                             int nkv, uint32_t &it, uint32_t k, int t, int q_rows, int pos,
-                                             int first_pos, int tok0, int head, bool &err) {
+__device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, int kv_tile0, int row_base, int piece,
+                                             uint32_t trow, uint32_t s_col, uint32_t o_col, uint64_t *s_full,
+                                             uint64_t *p_full, uint64_t *o_done, uint64_t *o_free, uint32_t &it,
+                                             uint32_t k, int t, int q_rows, int pos, int first_pos, int tok0, int head,
+                                             int hl, bool &err) {
     float m = -INFINITY, l = 0.f;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
     for (int j = 0; j < nkv; ++j, ++it) {
         if (!err && !mbar_wait(s_full, it & 1)) err = true;
         tc_fence_after();
-        const int kbase = 128 * j;
+        const int kbase = 128 * (kv_tile0 + j);  // first key of this step
         // only tiles that reach past the first query's position need the
         // causal mask (pos < n also covers the segment's length)
         const bool masked = kbase + 127 > first_pos;
@@ -300,6 +301,26 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, uint32_t tr
     tmem_ld_wait();
     tc_fence_before();
     mbar_arrive(o_free);
+    if (row_base >= 0) {
+        // shared-prefix tile: unnormalised O and (max, sum) become one
+        // partial of the decode row of this token and kv head (hl: the
+        // head's index within its kv group)
+        if (t < q_rows) {
+            const int G = p.group;
+            const int r = row_base + t * p.num_kv_heads;
+            const int slot = p.combine[p.rows[r].combine].piece_base + piece;
+            float *po = p.partial_o + ((size_t)slot * G + hl) * D;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    reinterpret_cast<float4 *>(po + 32 * i)[c] =
+                        make_float4(__uint_as_float(o[i][4 * c]), __uint_as_float(o[i][4 * c + 1]),
+                                    __uint_as_float(o[i][4 * c + 2]), __uint_as_float(o[i][4 * c + 3]));
+            p.partial_ml[(size_t)slot * G + hl] = make_float2(m, l);
+        }
+        return;
+    }
     const float inv = 1.f / l;
     if (t < q_rows) {
         __nv_bfloat16 *orow = p.out + ((size_t)(tok0 + t) * p.num_q_heads + head) * D;
@@ -332,7 +353,7 @@ __global__ void __launch_bounds__(256) stage_kernel(const __grid_constant__ Pref
     constexpr int kRowChunks = D / 8;
     const int kv = blockIdx.y;
     const StageTile st = p.stages[blockIdx.x];
-    const int n = p.seq_lens[st.seq];
+    const int n = st.n_keys;
     const int32_t *bt_row = p.block_tables + (size_t)st.seq * p.max_blocks_per_seq;
     const __nv_bfloat16 *cache = kv ? p.v_cache : p.k_cache;
     uint8_t *tile = p.staged + ((size_t)blockIdx.x * 2 + kv) * (128 * D * 2);
@@ -513,7 +534,7 @@ __global__ void __launch_bounds__(384, 1)
                 const bool two = tile.num_heads == 2;
                 const int nkv = tile.n_kv_tiles;
                 const int hA = tile.head;
-                const int tok0 = p.cu_seqlens_q[tile.seq] + tile.q_start;
+                const int tok0 = tile.row_base >= 0 ? tile.q_start : p.cu_seqlens_q[tile.seq] + tile.q_start;
                 if (ti > t_begin && !err && !mbar_wait(q_empty, (uint32_t)(ti - t_begin - 1) & 1)) err = true;
                 mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kTileBytes);
 #pragma unroll
@@ -522,7 +543,7 @@ __global__ void __launch_bounds__(384, 1)
                     if (two) tma_load_3d(sQB + s * 16384, &maps.q, q_full, 64 * s, hA + 1, tok0);
                 }
                 // staged tile kv_base + j: K then V, kTileBytes each
-                const uint8_t *kv_tiles = p.staged + (size_t)tile.kv_base * 2 * C::kTileBytes;
+                const uint8_t *kv_tiles = p.staged + (size_t)(tile.kv_base + tile.kv_tile0) * 2 * C::kTileBytes;
                 auto load_k = [&](int j) {
                     if (kuse >= (uint32_t)C::kKStages && !err &&
                         !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1))
@@ -561,16 +582,27 @@ __global__ void __launch_bounds__(384, 1)
         for (int ti = t_begin; ti < t_end; ++ti) {
             const PrefillTile tile = p.tiles[ti];
             if (!headA && tile.num_heads != 2) continue;
-            const int seq = tile.seq, q0 = tile.q_start;
-            const int tok0 = p.cu_seqlens_q[seq] + q0;
-            const int L = p.cu_seqlens_q[seq + 1] - p.cu_seqlens_q[seq];
-            const int n = p.seq_lens[seq];
-            const int q_rows = min(128, L - q0);
-            const int first_pos = n - L + q0;
-            const int pos = t < q_rows ? first_pos + t : 0;  // padding rows see key 0 only
-            softmax_tile<D>(p, trow, headA ? C::kSA : C::kSB, headA ? C::kOA : C::kOB, headA ? sA_full : sB_full,
-                            headA ? pA_full : pB_full, headA ? oA_done : oB_done, headA ? oA_free : oB_free,
-                            tile.n_kv_tiles, it, k, t, q_rows, pos, first_pos, tok0, tile.head + (headA ? 0 : 1), err);
+            int tok0, q_rows, first_pos, pos;
+            if (tile.row_base >= 0) {
+                // shared prefix: every query sees all keys < key_limit
+                tok0 = tile.q_start;
+                q_rows = tile.q_rows;
+                first_pos = tile.key_limit - 1;
+                pos = t < q_rows ? first_pos : 0;
+            } else {
+                const int seq = tile.seq, q0 = tile.q_start;
+                tok0 = p.cu_seqlens_q[seq] + q0;
+                const int L = p.cu_seqlens_q[seq + 1] - p.cu_seqlens_q[seq];
+                const int n = p.seq_lens[seq];
+                q_rows = min(128, L - q0);
+                first_pos = n - L + q0;
+                pos = t < q_rows ? first_pos + t : 0;  // padding rows see key 0 only
+            }
+            const int head = tile.head + (headA ? 0 : 1);
+            softmax_tile<D>(p, tile.n_kv_tiles, tile.kv_tile0, tile.row_base, tile.piece, trow,
+                            headA ? C::kSA : C::kSB, headA ? C::kOA : C::kOB, headA ? sA_full : sB_full,
+                            headA ? pA_full : pB_full, headA ? oA_done : oB_done, headA ? oA_free : oB_free, it, k, t,
+                            q_rows, pos, first_pos, tok0, head, head % p.group, err);
             ++k;
         }
     }

@@ -120,7 +120,7 @@ def test_plan_rebuild_in_place(lib):
     h = plan.handle
     d = dims_for(a)
     assert lib.pa_plan_build(a.cu_seqlens_q.ctypes.data_as(ctypes.c_void_p),
-                             a.seq_lens.ctypes.data_as(ctypes.c_void_p), ctypes.byref(d), 0,
+                             a.seq_lens.ctypes.data_as(ctypes.c_void_p), None, ctypes.byref(d), 0,
                              ctypes.byref(h)) == pa.PA_ERR_PLAN
 
 
@@ -141,7 +141,7 @@ def test_plan_rejects_bad_arguments(lib):
 
     def build(cu, sl, d):
         h = ctypes.c_void_p()          # NULL: ask for a new plan
-        st = lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p),
+        st = lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p), None,
                                ctypes.byref(d), -1, ctypes.byref(h))
         assert st == pa.PA_OK or not h.value
         lib.pa_plan_destroy(h)
@@ -165,8 +165,8 @@ def test_plan_rejects_bad_arguments(lib):
     assert build(cu, sl, d) == pa.PA_ERR_UNSUPPORTED                 # group 17
     d = dims_for(lay); d.max_blocks_per_seq = 2
     assert build(cu, sl, d) == pa.PA_ERR_SHAPE                       # table too narrow
-    assert lib.pa_plan_build(None, None, ctypes.byref(dims_for(lay)), -1, ctypes.byref(h)) == pa.PA_ERR_NULL
-    assert lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p),
+    assert lib.pa_plan_build(None, None, None, ctypes.byref(dims_for(lay)), -1, ctypes.byref(h)) == pa.PA_ERR_NULL
+    assert lib.pa_plan_build(cu.ctypes.data_as(ctypes.c_void_p), sl.ctypes.data_as(ctypes.c_void_p), None,
                              ctypes.byref(dims_for(lay)), -1, None) == pa.PA_ERR_NULL
 
 

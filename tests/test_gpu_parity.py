@@ -23,13 +23,16 @@ def dims_for(lay):
                    lay.head_dim, lay.num_blocks, lay.max_blocks_per_seq, 16)
 
 
-def run_step(batch):
-    """Scatter then attention on the GPU, as one forward step does."""
+def run_step(batch, with_tables=True):
+    """Scatter then attention on the GPU, as one forward step does (the plan
+    sees the host block tables, as bench.py's does, unless with_tables is
+    False)."""
     lay = batch.layout
     kc, vc = batch.k_cache.clone(), batch.v_cache.clone()
     bt, cu, sl, slots = batch.device_ints("cuda")
     pa.reshape_and_cache(batch.k, batch.v, slots, kc, vc)
-    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay))
+    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay),
+                   block_tables=lay.block_tables if with_tables else None)
     ws = pa.workspace_for(plan)
     out = torch.full_like(batch.q, float("nan"))
     pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws)
@@ -168,6 +171,35 @@ def test_prefill_tensor_core_all_rows(cuda_lib, case, q_gain):
     assert plan.info()["num_prefill_tiles"] > 0
     tok, want = oracle_subset(b, range(lay.num_seqs))
     assert_parity(gpu_rows(out, tok), want, f"prefill case {case} q_gain={q_gain} plan={plan.info()}")
+
+
+SHARED = [
+    # (q_lens, seq_lens, Hq, Hkv, D, shared blocks): runs of single-token
+    # segments on a shared prefix are attended to it by the prefill kernel
+    # (partials) and to the rest of their keys by the decode kernel
+    ([1] * 8, [320 + s for s in (1, 7, 16, 17, 90, 150, 200, 33)], 16, 2, 128, 20),  # 3 key tiles, last partial
+    ([1] * 6, [256 + s for s in (1, 2, 64, 65, 300, 9)], 12, 2, 64, 16),            # G = 6, two key tiles
+    ([1, 1, 1, 1, 1, 40, 1], [400, 401, 450, 700, 385, 424, 399], 8, 8, 128, 24),    # G = 1, prefill breaks the run
+    ([1] * 130, [640 + (7 * i) % 300 for i in range(130)], 8, 1, 64, 40),            # 130 tokens: two query chunks
+]
+
+
+@pytest.mark.parametrize("case", range(len(SHARED)))
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_shared_prefix_all_rows(cuda_lib, case, q_gain):
+    q_lens, seq_lens, Hq, Hkv, D, k = SHARED[case]
+    nb = sum(-(-s // 16) for s in seq_lens) + 64
+    lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, nb, seed=300 + case, shared_prefix_blocks=k)
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, plan = run_step(b)
+    info = plan.info()
+    assert info["num_prefix_groups"] == 1
+    tok, want = oracle_subset(b, range(lay.num_seqs))
+    assert_parity(gpu_rows(out, tok), want, f"shared case {case} q_gain={q_gain} plan={info}")
+    # the same step planned without the tables (no cascade) agrees too
+    _, _, out2, plan2 = run_step(b, with_tables=False)
+    assert plan2.info()["num_prefix_groups"] == 0
+    assert_parity(gpu_rows(out2, tok), want, f"shared case {case} without cascade")
 
 
 def test_split_rows_are_exercised(cuda_lib):
