@@ -319,8 +319,10 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         }
     }
     // Shared-prefix tiles: per group, chunk of up to 128 tokens, kv head,
-    // query-head pair and key split.  The key splits make enough tiles to
-    // fill the GPU without cutting a split below four 128-key tiles.
+    // query-head pair and key split.  The key splits make about one tile per
+    // SM without cutting a split below four 128-key tiles: more splits also
+    // mean more partials for every row to merge (B200: 4 splits of a
+    // 4096-key prefix over 32 base tiles beat 2 and 8).
     for (size_t k = 0; k < groups.size(); ++k) {
         const PrefixGroup &gr = groups[k];
         const int keys = gr.blocks * pa::kBlockSize;
@@ -328,7 +330,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         const int chunks = (int)cdiv(gr.nseg, pa::kPrefillTileM);
         const int base_tiles = chunks * Hkv * (int)cdiv(G, 2);
         const int splits = (int)std::max<int64_t>(
-            1, std::min<int64_t>(cdiv(nt, 4), cdiv(2 * (int64_t)p->num_sms, base_tiles)));
+            1, std::min<int64_t>(cdiv(nt, 4), (int64_t)p->num_sms / base_tiles));
         group_splits[k] = splits;
         const int base = (int)stages.size();
         for (int g = 0; g < Hkv; ++g)
