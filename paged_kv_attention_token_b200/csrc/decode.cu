@@ -225,10 +225,11 @@ __device__ __forceinline__ void attend_step(RowState<D, NT> &st, uint32_t stage,
 }
 
 // Merge the partials of a split row and write it: O = sum_j 2^(m_j - M) O_j /
-// sum_j 2^(m_j - M) l_j with M = max_j m_j.  Run by the warp that took the
-// row's last ticket; the partials are read through L2 (ld.cg), where the other
-// warps' fenced writes are visible, kMergeBatch partials at a time so that the
-// loads overlap instead of forming a chain.
+// sum_j 2^(m_j - M) l_j with M = max_j m_j, in one pass with a running max.
+// Run by the warp that took the row's last ticket; the partials are read
+// through L2 (ld.cg), where the other warps' fenced writes are visible,
+// kMergeBatch partials at a time so that the loads overlap instead of
+// forming a chain.
 template <int D>
 __device__ __noinline__ void merge_split_row(const DecodeParams &p, const CombineRow c, int token,
                                              int h0, int tid, int nthreads) {
@@ -238,17 +239,9 @@ __device__ __noinline__ void merge_split_row(const DecodeParams &p, const Combin
     for (int item = tid; item < G * (D / 8); item += nthreads) {
         const int head = item / (D / 8);
         const int chunk = item % (D / 8);
-        float M = -INFINITY;
-        for (int j0 = 0; j0 < n; j0 += kMergeBatch) {
-            float mj[kMergeBatch];
-#pragma unroll
-            for (int k = 0; k < kMergeBatch; ++k)
-                mj[k] = j0 + k < n ? __ldcg(&p.partial_ml[(size_t)(c.piece_base + j0 + k) * G + head]).x
-                                   : -INFINITY;
-#pragma unroll
-            for (int k = 0; k < kMergeBatch; ++k) M = fmaxf(M, mj[k]);
-        }
-        float den = 0.f;
+        // one pass: a batch's (max, sum) and O are loaded together and folded
+        // into a running max, sum and accumulator
+        float M = -INFINITY, den = 0.f;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j0 = 0; j0 < n; j0 += kMergeBatch) {
             float2 ml[kMergeBatch];
@@ -266,13 +259,21 @@ __device__ __noinline__ void merge_split_row(const DecodeParams &p, const Combin
                     lo[k] = hi[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+            float Mn = M;
+#pragma unroll
+            for (int k = 0; k < kMergeBatch; ++k) Mn = fmaxf(Mn, ml[k].x);
+            const float s = M == -INFINITY ? 0.f : exp2f(M - Mn);  // earlier batches, rescaled
+            den *= s;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] *= s;
 #pragma unroll
             for (int k = 0; k < kMergeBatch; ++k) {
-                const float w = exp2f(ml[k].x - M);  // 0 for the padding entries
+                const float w = exp2f(ml[k].x - Mn);  // 0 for the padding entries
                 den += w * ml[k].y;
                 acc[0] += w * lo[k].x; acc[1] += w * lo[k].y; acc[2] += w * lo[k].z; acc[3] += w * lo[k].w;
                 acc[4] += w * hi[k].x; acc[5] += w * hi[k].y; acc[6] += w * hi[k].z; acc[7] += w * hi[k].w;
             }
+            M = Mn;
         }
         const float inv = 1.f / den;
         uint4 o;

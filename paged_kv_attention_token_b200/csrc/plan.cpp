@@ -44,6 +44,12 @@ constexpr int64_t kTileOverheadSteps = 2;
 // q, the final write or merge) stay small against the streaming.
 constexpr int64_t kMinBlocksPerUnit = 4;
 
+// Cost, in blocks, charged at the end of every decode row when runs are cut:
+// finishing a row (the output write, or a partial, its ticket and often the
+// merge) and starting the next (its q) take about as long as streaming this
+// many blocks, so a run that crosses a row boundary gets fewer blocks.
+constexpr int64_t kRowCostBlocks = 4;
+
 // Cost model for running the prefill kernel beside the decode kernel on
 // disjoint SMs (B200 measurements): one 128-key step of a two-head tile
 // takes a CTA (one SM) ~2.9 us when the prefill kernel has a part of the
@@ -391,12 +397,17 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         tiles.swap(dealt);
     }
 
-    // Cut the decode rows' blocks into equal runs.
+    // Cut the decode rows' blocks into equal runs of cost: each row's
+    // blocks, then kRowCostBlocks of virtual cost, laid end to end.
     const int64_t R = (int64_t)rows.size();
-    std::vector<int64_t> prefix(R + 1, 0);
-    for (int64_t r = 0; r < R; ++r)
-        prefix[r + 1] = prefix[r] + cdiv(rows[r].n_keys, pa::kBlockSize) - rows[r].first_block;
-    const int64_t total = prefix[R];
+    std::vector<int64_t> prefix(R + 1, 0), nblocks(R, 0);
+    for (int64_t r = 0; r < R; ++r) {
+        nblocks[r] = cdiv(rows[r].n_keys, pa::kBlockSize) - rows[r].first_block;
+        prefix[r + 1] = prefix[r] + nblocks[r] + kRowCostBlocks;
+    }
+    const int64_t total_cost = prefix[R];
+    int64_t total = 0;  // real blocks
+    for (int64_t r = 0; r < R; ++r) total += nblocks[r];
     int64_t P = 0;
     if (total > 0) {
         const int64_t max_units = (int64_t)decode_sms * pa::decode_units_per_sm(d.head_dim);
@@ -407,11 +418,16 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     {
         int64_t r = 0;
         for (int64_t u = 0; u <= P; ++u) {
-            const int64_t f = P ? total * u / P : 0;
+            const int64_t f = P ? total_cost * u / P : 0;
             ustart[u] = f;
-            while (r < R && prefix[r + 1] <= f) ++r;  // row holding block f
-            units[u] = {(int32_t)r, (int32_t)(f - prefix[std::min(r, R)]) + (r < R ? rows[r].first_block : 0),
-                        r < R ? rows[r].seq : 0, r < R ? rows[r].n_keys : 0};
+            while (r < R && prefix[r + 1] <= f) ++r;  // row whose cost span holds f
+            int64_t rr = r, off = r < R ? f - prefix[r] : 0;
+            if (rr < R && off >= nblocks[rr]) {  // in the row's virtual cost: start the next row
+                ++rr;
+                off = 0;
+            }
+            units[u] = {(int32_t)rr, (int32_t)off + (rr < R ? rows[rr].first_block : 0),
+                        rr < R ? rows[rr].seq : 0, rr < R ? rows[rr].n_keys : 0};
         }
         units[P] = {(int32_t)R, 0, 0, 0};
     }
@@ -423,7 +439,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         for (int64_t r = 0; r < R; ++r) {
             while (u + 1 < P && ustart[u + 1] <= prefix[r]) ++u;  // unit of the first block
             int64_t v = u;
-            while (v + 1 < P && ustart[v + 1] <= prefix[r + 1] - 1) ++v;  // unit of the last block
+            while (v + 1 < P && ustart[v + 1] <= prefix[r] + nblocks[r] - 1) ++v;  // unit of the last block
             const int32_t count = (int32_t)(v - u + 1);
             // partials of the row's shared prefix (written by the prefill
             // kernel) come first
