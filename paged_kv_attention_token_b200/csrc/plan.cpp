@@ -48,7 +48,7 @@ constexpr int64_t kMinBlocksPerUnit = 4;
 // finishing a row (the output write, or a partial, its ticket and often the
 // merge) and starting the next (its q) take about as long as streaming this
 // many blocks, so a run that crosses a row boundary gets fewer blocks.
-constexpr int64_t kRowCostBlocks = 4;
+constexpr int64_t kRowCostBlocks = 8;
 
 // Cost model for running the prefill kernel beside the decode kernel on
 // disjoint SMs (B200 measurements): one 128-key step of a two-head tile

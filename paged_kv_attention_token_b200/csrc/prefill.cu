@@ -47,10 +47,8 @@
 //               scale*log2(e), moves its running max (and rescales its O row
 //               in TMEM) only when it grows by more than
 //               kPrefillRescaleThreshold, and writes P into the S columns.
-//               A quarter of the exponentials are evaluated on the FMA pipe
-//               (exp2_fma), the rest on the MUFU unit, whose 16 results per
-//               SM and clock would otherwise bound the tile rate.  At the
-//               end it reads its O row, divides by its sum and writes bf16.
+//               At the end it reads its O row, divides by its sum and
+//               writes bf16.
 // Every wait is on an mbarrier and bounded; on a timeout the kernel sets a
 // bit in the workspace status word and runs to the end without waiting,
 // after which TMEM is released.
@@ -136,42 +134,10 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
-}
-
-// 2^x for a pair, on the FMA pipe: x = i + f with i = round(x) and f in
-// [-1/2, 1/2]; 2^f from a cubic fitted (weighted least squares, relative
-// error) to 2^f on that interval: max relative error 7.5e-5 (~13.7 bits),
-// below the bf16 rounding P gets next.  2^i is added to the exponent field.
-// x is clamped to >= -125 so that the exponent never underflows: results
-// there are ~2^-125 instead of 0, which callers replace by 0 where a key is
-// masked.
-__device__ __forceinline__ void exp2_fma(uint64_t x2, float &e0, float &e1) {
-    constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
-    float x0, x1;
-    f2_split(x2, x0, x1);
-    x2 = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t r2 = f2(kRound, kRound);
-    const uint64_t t = f2_add(x2, r2);  // kRound + round(x): round(x) in the low bits
-    const uint64_t fr = f2_sub(x2, f2_sub(t, r2));
-    uint64_t p = f2_fma(f2(0.055171508f, 0.055171508f), fr, f2(0.24261114f, 0.24261114f));
-    p = f2_fma(p, fr, f2(0.69326103f, 0.69326103f));
-    p = f2_fma(p, fr, f2(0.99992806f, 0.99992806f));
-    float p0, p1, t0, t1;
-    f2_split(p, p0, p1);
-    f2_split(t, t0, t1);
-    // shifted by 23, the low bits of t's encoding (round(x) in two's
-    // complement) become the exponent increment; the bits above fall off
-    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Row max over 32 S columns; keys > pos excluded when `masked`.
@@ -187,30 +153,22 @@ __device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], float mx, bo
 }
 
 // P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; adds the
-// rounded values to lsum (as a packed pair of partial sums).  Pairs 3, 7,
-// 11 and 15 use exp2_fma, the others ex2.approx.
+// rounded values to lsum (as a packed pair of partial sums), so that the
+// sum matches the P the PV product uses.  (Evaluating part of the
+// exponentials on the FMA pipe with a polynomial was measured slower here:
+// the softmax is bound by issue and latency, not by the MUFU unit.)
 __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t &lsum,
                                           uint64_t scale2, uint64_t nm2, bool masked, int key0, int pos) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
-        float e0, e1;
-        if ((c & 3) == 3) {
-            exp2_fma(x, e0, e1);
-            if (masked) {
-                if (key0 + 2 * c > pos) e0 = 0.f;
-                if (key0 + 2 * c + 1 > pos) e1 = 0.f;
-            }
-        } else {
-            float x0, x1;
-            f2_split(x, x0, x1);
-            if (masked) {
-                if (key0 + 2 * c > pos) x0 = -INFINITY;
-                if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
-            }
-            e0 = fast_exp2(x0);
-            e1 = fast_exp2(x1);
+        float x0, x1;
+        f2_split(x, x0, x1);
+        if (masked) {
+            if (key0 + 2 * c > pos) x0 = -INFINITY;
+            if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
         }
+        const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
         pk[c] = pack_bf16x2(e0, e1);
         lsum = f2_add(lsum, f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
     }
