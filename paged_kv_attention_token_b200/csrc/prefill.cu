@@ -140,25 +140,34 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
-// Row max over 32 S columns; keys > pos excluded when `masked`.
-__device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], float mx, bool masked, int key0, int pos) {
+// Max over 32 S columns; keys > pos excluded when `masked`.  Two
+// independent chains, so that the reduction's latency is half its length.
+__device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], bool masked, int key0, int pos) {
+    float a = -INFINITY, b = -INFINITY;
     if (!masked) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) mx = max3f(mx, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        for (int c = 0; c < 32; c += 4) {
+            a = max3f(a, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+            b = max3f(b, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+        }
     } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, key0 + c <= pos ? __uint_as_float(r[c]) : -INFINITY);
+        for (int c = 0; c < 32; c += 2) {
+            a = fmaxf(a, key0 + c <= pos ? __uint_as_float(r[c]) : -INFINITY);
+            b = fmaxf(b, key0 + c + 1 <= pos ? __uint_as_float(r[c + 1]) : -INFINITY);
+        }
     }
-    return mx;
+    return fmaxf(a, b);
 }
 
-// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; adds the
-// rounded values to lsum (as a packed pair of partial sums), so that the
-// sum matches the P the PV product uses.  (Evaluating part of the
+// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; lsum gets
+// the sum of the rounded values (as a packed pair of partial sums), so that
+// the sum matches the P the PV product uses.  (Evaluating part of the
 // exponentials on the FMA pipe with a polynomial was measured slower here:
 // the softmax is bound by issue and latency, not by the MUFU unit.)
 __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t &lsum,
                                           uint64_t scale2, uint64_t nm2, bool masked, int key0, int pos) {
+    uint64_t sum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};  // two independent chains
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
@@ -170,8 +179,9 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk
         }
         const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
         pk[c] = pack_bf16x2(e0, e1);
-        lsum = f2_add(lsum, f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
+        sum[c & 1] = f2_add(sum[c & 1], f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
     }
+    lsum = f2_add(sum[0], sum[1]);
 }
 
 // Softmax of one head for one tile, one query row per thread (128 threads);
@@ -202,10 +212,8 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         tmem_ld32(trow + s_col + 96, s3);
         tmem_ld_wait();
         // row max of the raw scores (scale > 0 commutes with max)
-        float mx = chunk_max(s0, -INFINITY, masked, kbase, pos);
-        mx = chunk_max(s1, mx, masked, kbase + 32, pos);
-        mx = chunk_max(s2, mx, masked, kbase + 64, pos);
-        mx = chunk_max(s3, mx, masked, kbase + 96, pos);
+        float mx = fmaxf(fmaxf(chunk_max(s0, masked, kbase, pos), chunk_max(s1, masked, kbase + 32, pos)),
+                         fmaxf(chunk_max(s2, masked, kbase + 64, pos), chunk_max(s3, masked, kbase + 96, pos)));
         mx *= p.scale_log2;
         float alpha = 1.f;
         const bool rescale = mx > m + kPrefillRescaleThreshold;
@@ -216,17 +224,19 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         // P = 2^(s*scale - m) as bf16, written over the S columns (P chunk
         // i goes to columns 16 i .. 16 i + 15)
         const uint64_t nm2 = f2(-m, -m);
-        uint64_t lsum = f2(0.f, 0.f);
+        uint64_t lsum;
         {
             uint32_t pk[16];
-            chunk_exp(s0, pk, lsum, scale2, nm2, masked, kbase, pos);
+            uint64_t ls[4];  // per-chunk sums, added at the end
+            chunk_exp(s0, pk, ls[0], scale2, nm2, masked, kbase, pos);
             tmem_st16(trow + s_col, pk);
-            chunk_exp(s1, pk, lsum, scale2, nm2, masked, kbase + 32, pos);
+            chunk_exp(s1, pk, ls[1], scale2, nm2, masked, kbase + 32, pos);
             tmem_st16(trow + s_col + 16, pk);
-            chunk_exp(s2, pk, lsum, scale2, nm2, masked, kbase + 64, pos);
+            chunk_exp(s2, pk, ls[2], scale2, nm2, masked, kbase + 64, pos);
             tmem_st16(trow + s_col + 32, pk);
-            chunk_exp(s3, pk, lsum, scale2, nm2, masked, kbase + 96, pos);
+            chunk_exp(s3, pk, ls[3], scale2, nm2, masked, kbase + 96, pos);
             tmem_st16(trow + s_col + 48, pk);
+            lsum = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
         }
         float l0, l1;
         f2_split(lsum, l0, l1);
