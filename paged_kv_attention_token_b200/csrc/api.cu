@@ -188,6 +188,7 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.group = plan->group;
         p.max_blocks_per_seq = d.max_blocks_per_seq;
         p.scale_log2 = scale_log2;
+        p.defer_merge = 0;
     }
     PrefillParams pp{};
     if (plan->num_tiles > 0) {
@@ -235,10 +236,15 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (cudaStreamWaitEvent(side, fork, 0) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 1, side) != cudaSuccess) return PA_ERR_CUDA;
+        // shared-prefix partials are not ready while the decode kernel runs:
+        // it leaves every merge to the merge kernel after the join
+        p.defer_merge = plan->cascade ? 1 : 0;
         if (launch_decode(p, d.head_dim, side) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 2, side) != cudaSuccess || mark(trace, 3, side) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;  // prefill, not the join
         if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
+            return PA_ERR_CUDA;
+        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
             return PA_ERR_CUDA;
         if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
         return PA_OK;

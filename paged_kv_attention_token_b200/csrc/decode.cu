@@ -524,9 +524,11 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
                     }
                     if (g8 == 0) p.partial_ml[(size_t)slot * G + head] = make_float2(st.m[nt][e], st.l[nt][e]);
                 }
-            // publish the partial, take a ticket; the last warp of the row merges
+            // publish the partial, take a ticket; the last warp of the row
+            // merges (unless a separate merge kernel follows)
             __threadfence();
             __syncwarp();
+            if (p.defer_merge) return;
             int last = 0;
             const CombineRow c = p.combine[row.combine];
             if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.tickets - 1;
@@ -540,6 +542,19 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
         }
     });
     cp_async_wait<0>();  // nothing may still be landing when the warp exits
+}
+
+// Merges every combine row, one warp per row: used when the decode kernel
+// ran beside the kernel that writes a row's shared-prefix partials, so that
+// neither can merge.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ DecodeParams p, int num_combine) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ci = blockIdx.x * 4 + warp;
+    if (ci >= num_combine) return;
+    const CombineRow c = p.combine[ci];
+    const DecodeRow row = p.rows[c.row];
+    merge_split_row<D>(p, c, row.token, (c.row % p.num_kv_heads) * p.group, lane, 32);
 }
 
 template <int D, int NT>
@@ -564,6 +579,16 @@ cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
 int decode_units_per_sm(int head_dim) {
     return head_dim == 64 ? DecodeCfg<64, 1>::kWarps * DecodeCfg<64, 1>::kCtasPerSm
                           : DecodeCfg<128, 1>::kWarps * DecodeCfg<128, 1>::kCtasPerSm;
+}
+
+cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, cudaStream_t stream) {
+    if (num_combine == 0) return cudaSuccess;
+    const int grid = (num_combine + 3) / 4;
+    if (head_dim == 64)
+        merge_kernel<64><<<grid, 128, 0, stream>>>(p, num_combine);
+    else
+        merge_kernel<128><<<grid, 128, 0, stream>>>(p, num_combine);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream) {

@@ -28,6 +28,7 @@ struct DecodeParams {
     int group;
     int max_blocks_per_seq;
     float scale_log2;
+    int defer_merge;            // nonzero: split rows only write partials (merge_kernel follows)
 };
 
 cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t *slots,
@@ -36,6 +37,8 @@ cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t
                                      cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);
+// Merges all combine rows (after a decode launch with defer_merge).
+cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, cudaStream_t stream);
 
 struct PrefillParams {
     const __nv_bfloat16 *q;

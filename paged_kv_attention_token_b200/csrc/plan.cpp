@@ -37,8 +37,16 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Start/finish cost of a prefill tile in units of 128-key steps (Q load,
-// first S, output write-back), for the CTA assignment.
+// first S, output write-back), for the CTA assignment and the side-by-side
+// split.  Shared-prefix tiles are short (a few steps) and write fp32
+// partials; beside the decode kernel they cost more (B200 sweep of the
+// shared-prefix workload: 8 steps beat 2, 16, 24 and running serially).
 constexpr int64_t kTileOverheadSteps = 2;
+constexpr int64_t kPrefixTileOverheadSteps = 8;
+
+int64_t tile_cost(const pa::PrefillTile &t) {
+    return t.n_kv_tiles + (t.row_base >= 0 ? kPrefixTileOverheadSteps : kTileOverheadSteps);
+}
 
 // Fewest KV blocks one decode warp is given, so that its fixed costs (loading
 // q, the final write or merge) stay small against the streaming.
@@ -355,22 +363,20 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         p->prefill_pairs += (int64_t)gr.nseg * keys;
     }
     std::stable_sort(tiles.begin(), tiles.end(),
-                     [](const pa::PrefillTile &a, const pa::PrefillTile &b) {
-                         return a.n_kv_tiles > b.n_kv_tiles;
-                     });
+                     [](const pa::PrefillTile &a, const pa::PrefillTile &b) { return tile_cost(a) > tile_cost(b); });
     // Deal the tiles to persistent CTAs; each CTA's tiles become contiguous.
     // Decode KV bytes and prefill steps decide whether the two kernels share
     // the GPU side by side, and on how many SMs each runs.
     int64_t decode_blocks_all = 0;
     for (const pa::DecodeRow &r : rows) decode_blocks_all += cdiv(r.n_keys, pa::kBlockSize) - r.first_block;
     int64_t prefill_steps = 0;
-    for (const pa::PrefillTile &t : tiles) prefill_steps += t.n_kv_tiles + kTileOverheadSteps;
-    // the decode kernel merges shared-prefix partials, so it follows the
-    // prefill kernel when there are any
+    for (const pa::PrefillTile &t : tiles) prefill_steps += tile_cost(t);
+    // With shared prefixes the decode rows merge partials of the prefill
+    // kernel: the decode kernel follows it, or runs beside it and leaves all
+    // merging to a merge kernel after both.
     p->cascade = !groups.empty();
     p->num_prefix_groups = (int32_t)groups.size();
-    p->overlap_sms = p->cascade ? 0 : overlap_split(p->num_sms, prefill_steps,
-                                   decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2);
+    p->overlap_sms = overlap_split(p->num_sms, prefill_steps, decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2);
     const int prefill_sms = p->overlap_sms > 0 ? p->overlap_sms : p->num_sms;
     const int decode_sms = p->num_sms - p->overlap_sms;
     const int grid = (int)std::min<size_t>(tiles.size(), (size_t)prefill_sms);
@@ -384,7 +390,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
             Load l = heap.top();
             heap.pop();
             per[l.second].push_back((int32_t)t);
-            l.first += tiles[t].n_kv_tiles + kTileOverheadSteps;
+            l.first += tile_cost(tiles[t]);
             heap.push(l);
         }
         std::vector<pa::PrefillTile> dealt;
