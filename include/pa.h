@@ -92,7 +92,10 @@ typedef struct {
  *                         tokens share a slot (precondition)
  *   d_k_cache, d_v_cache  device [NB][16][Hkv][D] bf16, written in place
  *   dims                  host; num_seqs, num_q_heads, max_blocks_per_seq unused
- * T == 0 queues nothing and returns PA_OK.
+ * T == 0 queues nothing and returns PA_OK.  The kernel lets a
+ * programmatically launched kernel queued after it (the attention call's
+ * decode kernel) start setting up early; that kernel still reads the caches
+ * only after this one has completed.
  */
 int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot_mapping,
                          void *d_k_cache, void *d_v_cache, const pa_dims *dims,
@@ -212,8 +215,13 @@ void pa_plan_destroy(pa_plan *plan);
  *                   in flight at once need two workspaces.
  * After a call that reported an error, rebuild the plan (its merge tickets
  * may be left taken) and reset the workspace's status word.
- * The call makes `stream` wait for the plan's upload, then queues its
- * kernels; nothing is copied from the host.
+ * The call makes `stream` wait for the plan's upload (no wait once the host
+ * has seen it complete), then queues its kernels; nothing is copied from the
+ * host.  The decode kernel is launched with programmatic stream
+ * serialization: its blocks may start while the kernel queued before it on
+ * `stream` is still running, read only the plan's tables until that kernel
+ * has completed (griddepcontrol.wait), and then everything else.  Stream
+ * order is therefore kept for all caller data.
  * Errors: PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_UNSUPPORTED,
  * PA_ERR_PLAN, PA_ERR_WORKSPACE, PA_ERR_CUDA.
  */

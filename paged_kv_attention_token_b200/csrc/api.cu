@@ -164,9 +164,19 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const uint8_t *tb = static_cast<const uint8_t *>(plan->d_tables);
     if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
-    // the upload queued by the plan's build (usually long done)
-    if (cudaStreamWaitEvent(stream, static_cast<cudaEvent_t>(plan->upload_event), 0) != cudaSuccess)
-        return PA_ERR_CUDA;
+    // the upload queued by the plan's build (usually long done: then no
+    // stream wait, which keeps the decode kernel's programmatic launch
+    // directly behind the caller's previous kernel)
+    {
+        cudaEvent_t up = static_cast<cudaEvent_t>(plan->upload_event);
+        const cudaError_t qs = cudaEventQuery(up);
+        if (qs == cudaErrorNotReady) {
+            if (cudaPeekAtLastError() == cudaErrorNotReady) cudaGetLastError();
+            if (cudaStreamWaitEvent(stream, up, 0) != cudaSuccess) return PA_ERR_CUDA;
+        } else if (qs != cudaSuccess) {
+            return PA_ERR_CUDA;
+        }
+    }
     const float scale_log2 = scale * kLog2e;
     DecodeParams p{};
     if (plan->num_units > 0) {

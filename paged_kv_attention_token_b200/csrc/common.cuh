@@ -11,6 +11,19 @@ namespace pa {
 constexpr unsigned kFullMask = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running; grid_dependency_wait returns once that kernel has completed and
+// its writes are visible (at once when the launch had no such attribute).
+// Everything a kernel reads that the caller's earlier work may have written
+// (q, the caches, block tables, lengths, the workspace) is read after it.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream, if launched with that attribute, start
+// its blocks now (they still wait for this grid's completion before reading).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 16-byte read-only load that does not allocate in L1 (streamed KV data).
 __device__ __forceinline__ uint4 ld_stream16(const void *p) {
     uint4 r;

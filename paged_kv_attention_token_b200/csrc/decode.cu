@@ -417,14 +417,18 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
     const uint32_t ring = smem_u32(smem) + warp * S * C::kStageBytes;
     const int Hkv = p.num_kv_heads;
     const DecodeUnit run_end = p.units[unit + 1];
+    const DecodeUnit first = p.units[unit];
     const CopyPattern<D> cpat(lane, Hkv * D);
+    // the plan's tables are ready before the launch; the caller's data may be
+    // written by the kernel before this one (programmatic launch)
+    grid_dependency_wait();
 
     // Load cursor: this warp's next step to copy; S-1 steps run ahead.
     LoadCursor lc;
     {
         // the unit carries its first row's segment and length: the first
         // copies need no read of the row table
-        const DecodeUnit st = p.units[unit];
+        const DecodeUnit &st = first;
         lc.r = st.row;
         lc.b = st.block;
         lc.done = st.row > run_end.row || (st.row == run_end.row && st.block >= run_end.block);
@@ -570,8 +574,20 @@ cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_relaxed);
     }
-    decode_kernel<D, NT><<<(p.num_units + C::kWarps - 1) / C::kWarps, C::kThreads, C::kSmemBytes, stream>>>(p);
-    return cudaGetLastError();
+    // programmatic launch: the CTAs may become resident and read their work
+    // units while the kernel before them (usually the cache scatter) ends
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((p.num_units + C::kWarps - 1) / C::kWarps);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<D, NT>, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

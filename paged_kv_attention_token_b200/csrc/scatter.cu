@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4 *__restrict__ k, const uint4 *__restrict__ v, const int64_t *__restrict__ slots,
     uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, int64_t num_chunks,
     int chunks_per_token, int64_t num_slots) {
+    // an attention kernel queued next may set up while the copy runs
+    grid_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
         const int64_t t = c / chunks_per_token;
