@@ -328,8 +328,8 @@ def run_ours(args):
     ws = pa.workspace_for(plan0, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    # scatter, split-KV decode (split rows are merged inside it), prefill
-    launches_per_step = 1 + (1 if info["num_decode_units"] else 0) + (1 if info["num_prefill_tiles"] else 0)
+    # the scatter, then the kernels the attention call launches (plan info)
+    launches_per_step = (1 if lay.num_tokens else 0) + info["attention_launches"]  # scatter + attention
 
     # two plans rebuilt in turn, as an engine keeps them across steps
     plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt), pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt)]

@@ -168,13 +168,14 @@ typedef struct {
     int32_t num_prefill_tiles;    /* (128-query tile, query-head pair) items */
     int64_t decode_kv_blocks;     /* sum over decode rows of ceil(keys / 16) */
     int64_t prefill_causal_pairs; /* (query, visible key) pairs per query head */
-    uint64_t table_bytes;         /* plan tables copied into the workspace per call */
+    uint64_t table_bytes;         /* the plan's device tables (uploaded once per build) */
     uint64_t workspace_bytes;     /* = pa_plan_workspace_bytes */
     int32_t num_staged_kv_tiles;  /* 128-key K/V tiles of prefill segments gathered
                                      into the workspace (per kv head) */
     int32_t num_prefill_ctas;     /* persistent CTAs of the prefill kernel */
     int32_t num_prefix_groups;    /* shared-prefix runs found (h_block_tables given) */
-    int32_t reserved;
+    int32_t attention_launches;   /* kernels one pa_attention_varlen call launches
+                                     (decode, staging, prefill, merge) */
 } pa_plan_info;
 int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
 

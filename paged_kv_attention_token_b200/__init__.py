@@ -66,7 +66,7 @@ class PlanInfo(ctypes.Structure):
                 ("decode_kv_blocks", ctypes.c_int64), ("prefill_causal_pairs", ctypes.c_int64),
                 ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
                 ("num_staged_kv_tiles", ctypes.c_int32), ("num_prefill_ctas", ctypes.c_int32),
-                ("num_prefix_groups", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("num_prefix_groups", ctypes.c_int32), ("attention_launches", ctypes.c_int32)]
 
     def as_dict(self):
         return {n: int(getattr(self, n)) for n, _ in self._fields_}

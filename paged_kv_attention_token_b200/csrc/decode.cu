@@ -510,6 +510,8 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
                     }
                 }
         } else {
+            // the row's merge entry, loaded while the partial is written
+            const CombineRow c = p.combine[row.combine];
             const int slot = row.slot_base + unit;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -534,7 +536,6 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
             __syncwarp();
             if (p.defer_merge) return;
             int last = 0;
-            const CombineRow c = p.combine[row.combine];
             if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.tickets - 1;
             last = __shfl_sync(kFullMask, last, 0);
             if (last) {

@@ -535,7 +535,12 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     info->num_staged_kv_tiles = p->num_stages;
     info->num_prefill_ctas = p->num_prefill_ctas;
     info->num_prefix_groups = p->num_prefix_groups;
-    info->reserved = 0;
+    // as pa_attention_varlen launches them: the decode kernel; staging and
+    // prefill; the merge kernel when shared-prefix tiles run beside decode
+    const bool side_by_side = p->overlap_sms > 0 && p->num_units > 0 && p->num_tiles > 0;
+    info->attention_launches = (p->num_units > 0 ? 1 : 0) + (p->num_tiles > 0 ? 1 : 0) +
+                               (p->num_tiles > 0 && p->num_stages > 0 ? 1 : 0) +
+                               (side_by_side && p->cascade && p->num_combine > 0 ? 1 : 0);
     return PA_OK;
 }
 

@@ -160,14 +160,12 @@ __device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], bool masked,
     return fmaxf(a, b);
 }
 
-// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; lsum gets
-// the sum of the rounded values (as a packed pair of partial sums), so that
-// the sum matches the P the PV product uses.  (Evaluating part of the
-// exponentials on the FMA pipe with a polynomial was measured slower here:
-// the softmax is bound by issue and latency, not by the MUFU unit.)
-__device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t &lsum,
-                                          uint64_t scale2, uint64_t nm2, bool masked, int key0, int pos) {
-    uint64_t sum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};  // two independent chains
+// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs.
+// (Evaluating part of the exponentials on the FMA pipe with a polynomial,
+// or all of them as f16 pairs, was measured slower here: the softmax is
+// bound by the latency and count of its instructions, not by the MUFU unit.)
+__device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t scale2,
+                                          uint64_t nm2, bool masked, int key0, int pos) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
@@ -179,9 +177,27 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk
         }
         const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
         pk[c] = pack_bf16x2(e0, e1);
-        sum[c & 1] = f2_add(sum[c & 1], f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
     }
-    lsum = f2_add(sum[0], sum[1]);
+}
+
+// Sum of the 32 rounded values of a P chunk (as a packed pair of partial
+// sums), so that the row sum matches the P the PV product uses.  Two
+// independent chains.
+__device__ __forceinline__ uint64_t chunk_sum(const uint32_t (&pk)[16]) {
+    uint64_t sum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+        sum[c & 1] = f2_add(sum[c & 1], f2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
+    return f2_add(sum[0], sum[1]);
+}
+
+// Ties 16 registers to this point of the program (volatile asm keeps its
+// order), so that work on them is not scheduled before it.
+__device__ __forceinline__ void regs_after(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]));
 }
 
 // Softmax of one head for one tile, one query row per thread (128 threads);
@@ -224,23 +240,15 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         // P = 2^(s*scale - m) as bf16, written over the S columns (P chunk
         // i goes to columns 16 i .. 16 i + 15)
         const uint64_t nm2 = f2(-m, -m);
-        uint64_t lsum;
-        {
-            uint32_t pk[16];
-            uint64_t ls[4];  // per-chunk sums, added at the end
-            chunk_exp(s0, pk, ls[0], scale2, nm2, masked, kbase, pos);
-            tmem_st16(trow + s_col, pk);
-            chunk_exp(s1, pk, ls[1], scale2, nm2, masked, kbase + 32, pos);
-            tmem_st16(trow + s_col + 16, pk);
-            chunk_exp(s2, pk, ls[2], scale2, nm2, masked, kbase + 64, pos);
-            tmem_st16(trow + s_col + 32, pk);
-            chunk_exp(s3, pk, ls[3], scale2, nm2, masked, kbase + 96, pos);
-            tmem_st16(trow + s_col + 48, pk);
-            lsum = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
-        }
-        float l0, l1;
-        f2_split(lsum, l0, l1);
-        l = l * alpha + (l0 + l1);
+        uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
+        chunk_exp(s0, pk0, scale2, nm2, masked, kbase, pos);
+        tmem_st16(trow + s_col, pk0);
+        chunk_exp(s1, pk1, scale2, nm2, masked, kbase + 32, pos);
+        tmem_st16(trow + s_col + 16, pk1);
+        chunk_exp(s2, pk2, scale2, nm2, masked, kbase + 64, pos);
+        tmem_st16(trow + s_col + 32, pk2);
+        chunk_exp(s3, pk3, scale2, nm2, masked, kbase + 96, pos);
+        tmem_st16(trow + s_col + 48, pk3);
         // O_X is stable: S_Xj completing implies PV_X(j-1) completed; PV_Xj
         // waits for p_full.  TMEM loads and stores are warp-collective, so
         // the warp rescales if any lane needs it (alpha = 1 for the others).
@@ -258,6 +266,15 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
+        // the row sum, off the path that hands P to the tensor cores
+        regs_after(pk0);
+        regs_after(pk1);
+        regs_after(pk2);
+        regs_after(pk3);
+        const uint64_t lsum = f2_add(f2_add(chunk_sum(pk0), chunk_sum(pk1)), f2_add(chunk_sum(pk2), chunk_sum(pk3)));
+        float l0, l1;
+        f2_split(lsum, l0, l1);
+        l = l * alpha + (l0 + l1);
     }
     if (!err && !mbar_wait(o_done, k & 1)) err = true;
     tc_fence_after();

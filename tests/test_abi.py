@@ -203,3 +203,17 @@ def test_status_strings(lib):
     for s in range(-9, 1):
         assert pa.status_string(s)
     assert pa.status_string(-100) == "unknown status"
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_attention_launch_count(lib, name):
+    # decode kernel; staging + prefill; the merge kernel only when
+    # shared-prefix tiles run beside the decode kernel
+    lay = W.layout(name)
+    info = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay), device=-1,
+                   block_tables=lay.block_tables).info()
+    base = (info["num_decode_units"] > 0) + 2 * (info["num_prefill_tiles"] > 0)
+    assert base <= info["attention_launches"] <= base + (info["num_prefix_groups"] > 0)
+    if name == "prefix_llama3_70b_b128":
+        # 128 decodes on a 4096-token prefix: prefix tiles beside the suffix decode
+        assert info["num_prefix_groups"] == 1 and info["attention_launches"] == 4
