@@ -4,9 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one pass of the whole hot path over one batch: the host work
-partition (pa_plan_build), the cache write (pa_reshape_and_cache) and varlen
-paged attention (pa_attention_varlen: split-KV decode kernel + combine, and the
-tensor-core prefill kernel when the batch holds long segments).  Inputs are
+partition (pa_plan_build), then the cache write and varlen paged attention in
+one call (pa_reshape_and_attention: the scatter kernel, the split-KV decode
+kernel + combine, and the tensor-core prefill kernel when the batch holds long
+segments; with --two-calls, pa_reshape_and_cache then pa_attention_varlen).  Inputs are
 seeded and synthetic with the shapes of the named workload (model names give
 attention shapes only; no weights).  Default workload: 64 decodes with the
 TinyLlama-1.1B attention shape.
@@ -343,9 +344,13 @@ def run_ours(args):
         plan_s = time.perf_counter() - t0
         if ev is not None:
             ev[0].record(stream)
-        pa.reshape_and_cache(batch.k, batch.v, slots, kc, vc, stream=stream)
-        pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws,
-                            stream=stream, trace=trace)
+        if trace is not None or args.two_calls:  # the traced entry point is the two-call one
+            pa.reshape_and_cache(batch.k, batch.v, slots, kc, vc, stream=stream)
+            pa.attention_varlen(batch.q, kc, vc, bt, cu, sl, batch.scale, out, plan, ws,
+                                stream=stream, trace=trace)
+        else:
+            pa.reshape_and_attention(batch.k, batch.v, slots, batch.q, kc, vc, bt, cu, sl, batch.scale, out,
+                                     plan, ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         return plan, plan_s
@@ -467,9 +472,14 @@ def run_ours(args):
             for n in host:
                 dev_in[n].copy_(host[n], non_blocking=True)
             plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims, h_bt)
-            pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)
-            pa.attention_varlen(dev_in["q"], kc, vc, dev_in["bt"], dev_in["cu"], dev_in["sl"],
-                                batch.scale, out, plan, ws, stream=stream)
+            if args.two_calls:
+                pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)
+                pa.attention_varlen(dev_in["q"], kc, vc, dev_in["bt"], dev_in["cu"], dev_in["sl"],
+                                    batch.scale, out, plan, ws, stream=stream)
+            else:
+                pa.reshape_and_attention(dev_in["k"], dev_in["v"], dev_in["slots"], dev_in["q"], kc, vc,
+                                         dev_in["bt"], dev_in["cu"], dev_in["sl"], batch.scale, out, plan, ws,
+                                         stream=stream)
             out_host.copy_(out, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
@@ -505,6 +515,8 @@ def run_ours(args):
                        "tokens_per_step": lay.num_tokens,
                        "l2": "flushed before every timed step (1 GiB write, outside the events)",
                        "plan_us_host": 1e6 * statistics.median(plan_times),
+                       "step_api": ("pa_reshape_and_cache + pa_attention_varlen" if args.two_calls
+                                    else "pa_reshape_and_attention"),
                        "stages_ms": {"plan_wait": wait_ms, "decode": dec_ms, "combine": comb_ms,
                                      "prefill": prefill_ms,
                                      "note": "separate traced passes; event records add GPU time"},
@@ -534,6 +546,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="step through pa_reshape_and_cache + pa_attention_varlen instead of the fused call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

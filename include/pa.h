@@ -259,6 +259,33 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
                            size_t workspace_bytes, void *stream, const pa_trace *trace);
 
 /*
+ * One forward step's cache write and attention in one call: the work of
+ * pa_reshape_and_cache(d_k, d_v, d_slot_mapping, ...) followed by
+ * pa_attention_varlen(...), with the same arguments, outputs and errors
+ * (the caches are written exactly as pa_reshape_and_cache writes them; out
+ * equals pa_attention_varlen's bit for bit).  Cache write and attention
+ * overlap: the decode kernel starts behind the scatter kernel by
+ * programmatic launch and reads the keys of this step's own tokens from
+ * d_k / d_v instead of their cache slots ("vLLM 学习笔记 01" §1.6: each new
+ * token's K/V go to the slot its slot mapping names, and attention reads
+ * them there; here the decode rows take the same values before they land).
+ * Precondition (besides those of both calls): every token t of segment i at
+ * position p = seq_len - q_len + j has slot_mapping[t] ==
+ * block_tables[i][p / 16] * 16 + p % 16, i.e. the slot mapping and the block
+ * tables describe the same cache positions.
+ *   d_k, d_v         device [T][Hkv][D] bf16: this step's K/V, read
+ *   d_slot_mapping   device [T] int64
+ *   the rest         as pa_attention_varlen; d_k_cache / d_v_cache written
+ * Checks of both calls run before anything is queued.
+ */
+int pa_reshape_and_attention(const void *d_k, const void *d_v, const int64_t *d_slot_mapping,
+                             const void *d_q, void *d_k_cache, void *d_v_cache,
+                             const int32_t *d_block_tables, const int32_t *d_cu_seqlens_q,
+                             const int32_t *d_seq_lens, float scale, void *d_out, const pa_dims *dims,
+                             const pa_plan *plan, void *d_workspace, size_t workspace_bytes,
+                             void *stream);
+
+/*
  * Status word of a workspace: waits for `stream`, then copies the word to
  * *status.  0 means no error; bit 0 means some wait inside a kernel gave up
  * after about a second (the kernels never block longer, and the affected

@@ -93,6 +93,7 @@ def load_library():
             "pa_attention_varlen": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P]),
             "pa_attention_varlen_ex": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P, P]),
             "pa_attention_varlen_noalloc": (I, [P, P, P, P, P, P, F, P, DP, P, P]),
+            "pa_reshape_and_attention": (I, [P, P, P, P, P, P, P, P, P, F, P, DP, P, P, SZ, P]),
             "pa_noalloc_scratch_bytes": (SZ, []),
             "pa_workspace_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "pa_workspace_reset": (I, [P, P, P]),
@@ -299,6 +300,36 @@ def attention_varlen(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, 
     else:
         trace.arm(stream if stream is not None else torch.cuda.current_stream())
         _check(lib.pa_attention_varlen_ex(*args, ctypes.byref(trace)), "pa_attention_varlen_ex")
+    return out
+
+
+def reshape_and_attention(k, v, slot_mapping, q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens,
+                          scale, out, plan: Plan, workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """A step's cache write and attention in one call (pa_reshape_and_attention):
+    writes the caches like reshape_and_cache and out like attention_varlen."""
+    lib = load_library()
+    d = plan.dims
+    bf = torch.bfloat16
+    if tuple(q.shape) != (d.num_tokens, d.num_q_heads, d.head_dim) or out.shape != q.shape:
+        raise PaError(PA_ERR_SHAPE, "q/out shape does not match the plan")
+    if tuple(k.shape) != (d.num_tokens, d.num_kv_heads, d.head_dim) or v.shape != k.shape:
+        raise PaError(PA_ERR_SHAPE, "k/v shape does not match the plan")
+    if tuple(slot_mapping.shape) != (d.num_tokens,):
+        raise PaError(PA_ERR_SHAPE, "slot_mapping must be [T]")
+    if tuple(k_cache.shape) != (d.num_blocks, d.block_size, d.num_kv_heads, d.head_dim) or \
+            v_cache.shape != k_cache.shape:
+        raise PaError(PA_ERR_SHAPE, "cache shape does not match the plan")
+    if tuple(block_tables.shape) != (d.num_seqs, d.max_blocks_per_seq):
+        raise PaError(PA_ERR_SHAPE, "block_tables shape does not match the plan")
+    if workspace.dtype != torch.uint8:
+        raise PaError(PA_ERR_DTYPE, "workspace must be uint8")
+    _check(lib.pa_reshape_and_attention(
+        _dev_ptr(k, "k", bf), _dev_ptr(v, "v", bf), _dev_ptr(slot_mapping, "slot_mapping", torch.int64),
+        _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf), _dev_ptr(v_cache, "v_cache", bf),
+        _dev_ptr(block_tables, "block_tables", torch.int32), _dev_ptr(cu_seqlens_q, "cu_seqlens_q", torch.int32),
+        _dev_ptr(seq_lens, "seq_lens", torch.int32), ctypes.c_float(scale), _dev_ptr(out, "out", bf),
+        ctypes.byref(d), plan.handle, _dev_ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel()),
+        _stream_ptr(stream)), "pa_reshape_and_attention")
     return out
 
 

@@ -132,11 +132,12 @@ extern "C" int pa_attention_varlen(const void *q, const void *k_cache, const voi
                                   out, dims, plan, workspace, workspace_bytes, stream_, nullptr);
 }
 
-extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const void *v_cache,
-                                      const int32_t *block_tables, const int32_t *cu_seqlens_q,
-                                      const int32_t *seq_lens, float scale, void *out,
-                                      const pa_dims *dims, const pa_plan *plan, void *workspace,
-                                      size_t workspace_bytes, void *stream_, const pa_trace *trace) {
+namespace {
+// Host checks of an attention call: PA_OK when it may be queued (or when
+// there is nothing to do: T == 0).
+int check_attention(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    const int32_t *cu_seqlens_q, const int32_t *seq_lens, const void *out, const pa_dims *dims,
+                    const pa_plan *plan, const void *workspace, size_t workspace_bytes) {
     int st = check_common_dims(dims);
     if (st != PA_OK) return st;
     if (!plan) return PA_ERR_NULL;
@@ -154,12 +155,23 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return PA_ERR_ALIGN;
     const WorkspaceLayout &w = plan->ws;
-    const TableLayout &tl = plan->tl;
     if (!workspace || workspace_bytes < w.total) return PA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
     // the plan's tables live on its device
     int cur = -1;
     if (!plan->d_tables || cudaGetDevice(&cur) != cudaSuccess || cur != plan->device) return PA_ERR_PLAN;
+    return PA_OK;
+}
+
+// Queues the attention kernels of a checked call.  k_new / v_new (a fused
+// step, right behind the step's own scatter on `stream_`): the decode kernel
+// reads this step's keys from them.
+int queue_attention(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    const int32_t *cu_seqlens_q, const int32_t *seq_lens, float scale, void *out,
+                    const pa_dims &d, const pa_plan *plan, void *workspace, void *stream_, const pa_trace *trace,
+                    const void *k_new, const void *v_new) {
+    const WorkspaceLayout &w = plan->ws;
+    const TableLayout &tl = plan->tl;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const uint8_t *tb = static_cast<const uint8_t *>(plan->d_tables);
@@ -199,6 +211,9 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         p.max_blocks_per_seq = d.max_blocks_per_seq;
         p.scale_log2 = scale_log2;
         p.defer_merge = 0;
+        p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+        p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+        p.wait_first = 1;
     }
     PrefillParams pp{};
     if (plan->num_tiles > 0) {
@@ -270,6 +285,8 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
         return PA_OK;
     } else {
         if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+        // right behind the step's own scatter (fused step, no trace events)
+        p.wait_first = k_new != nullptr && !trace ? 0 : 1;
         if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess ||
             mark(trace, 4, stream) != cudaSuccess)
@@ -283,6 +300,42 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
     // the plan's next build waits for this
     if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
     return PA_OK;
+}
+}  // namespace
+
+extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const void *v_cache,
+                                      const int32_t *block_tables, const int32_t *cu_seqlens_q,
+                                      const int32_t *seq_lens, float scale, void *out,
+                                      const pa_dims *dims, const pa_plan *plan, void *workspace,
+                                      size_t workspace_bytes, void *stream, const pa_trace *trace) {
+    const int st = check_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, out, dims, plan,
+                                   workspace, workspace_bytes);
+    if (st != PA_OK || dims->num_tokens == 0) return st;
+    return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, *dims, plan,
+                           workspace, stream, trace, nullptr, nullptr);
+}
+
+extern "C" int pa_reshape_and_attention(const void *k, const void *v, const int64_t *slot_mapping,
+                                        const void *q, void *k_cache, void *v_cache,
+                                        const int32_t *block_tables, const int32_t *cu_seqlens_q,
+                                        const int32_t *seq_lens, float scale, void *out, const pa_dims *dims,
+                                        const pa_plan *plan, void *workspace, size_t workspace_bytes,
+                                        void *stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (dims->num_tokens > 0) {
+        if (!k || !v || !slot_mapping) return PA_ERR_NULL;
+        if (!aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)) return PA_ERR_ALIGN;
+    }
+    const int st = check_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, out, dims, plan,
+                                   workspace, workspace_bytes);
+    if (st != PA_OK || dims->num_tokens == 0) return st;
+    const pa_dims &d = *dims;
+    if (launch_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
+                                 (int64_t)d.num_blocks * d.block_size, current_sm_count(),
+                                 static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, d, plan,
+                           workspace, stream, nullptr, k, v);
 }
 
 extern "C" int pa_workspace_reset(void *workspace, const pa_plan *plan, void *stream_) {

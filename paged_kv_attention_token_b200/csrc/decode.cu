@@ -302,13 +302,17 @@ struct LoadCursor {
     int r, b, bend, nblk, g;
     const int32_t *bt_row;
     int bt_base, bt_val;
+    int n_keys, token, n_new;  // the row's keys, its query token and how many keys are new
     bool done;
 };
 
 __device__ __forceinline__ void cursor_set_row(const DecodeParams &p, const DecodeUnit &end, LoadCursor &c,
-                                               int seq, int n_keys) {
+                                               int seq, int n_keys, int token, int n_new) {
     c.bt_row = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
     c.nblk = (n_keys + 15) >> 4;
+    c.n_keys = n_keys;
+    c.token = token;
+    c.n_new = n_new;
     c.bend = (c.r == end.row) ? end.block : c.nblk;
     c.g = c.r % p.num_kv_heads;
     c.bt_base = -1;
@@ -329,7 +333,7 @@ __device__ __forceinline__ void cursor_enter_row(const DecodeParams &p, const De
         return;
     }
     c.b = row.first_block;
-    cursor_set_row(p, end, c, row.seq, row.n_keys);
+    cursor_set_row(p, end, c, row.seq, row.n_keys, row.token, row.n_new);
 }
 
 __device__ __forceinline__ int cursor_block_id(LoadCursor &c, int b, int lane) {
@@ -360,6 +364,9 @@ struct CopyPattern {
 };
 
 // Copies the blocks of the cursor's step into a stage and moves the cursor on.
+// With p.k_new (a fused scatter and attention step), the keys this step
+// writes are copied from k_new / v_new, the step's own K/V input, instead of
+// from cache slots the scatter may not have written yet.
 template <int D, int NB>
 __device__ __forceinline__ void issue_step(const DecodeParams &p, const DecodeUnit &end, LoadCursor &c,
                                            const CopyPattern<D> &cp, uint32_t stage, int lane) {
@@ -373,10 +380,31 @@ __device__ __forceinline__ void issue_step(const DecodeParams &p, const DecodeUn
         const __nv_bfloat16 *kb = p.k_cache + base;
         const __nv_bfloat16 *vb = p.v_cache + base;
         const uint32_t st = stage + nb * kBlockBytes;
+        const int key0 = 16 * (c.b + nb);
+        const int first_new = c.n_keys - c.n_new;
+        if (p.k_new != nullptr && key0 + 16 > first_new) {
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-            cp_async16(st + cp.dst[i], kb + cp.src[i]);
-            cp_async16(st + (D / 64) * 2048 + cp.dst[i], vb + cp.src[i]);
+            for (int i = 0; i < D / 16; ++i) {
+                const int cidx = lane + 32 * i;
+                const int key = key0 + cidx / (D / 8);
+                const __nv_bfloat16 *ks = kb + cp.src[i];
+                const __nv_bfloat16 *vs = vb + cp.src[i];
+                if (key >= first_new && key < c.n_keys) {
+                    // token of key: the row's query token is its last key
+                    const size_t o = ((size_t)(c.token - (c.n_keys - 1 - key)) * p.num_kv_heads + c.g) * D +
+                                     8 * (cidx % (D / 8));
+                    ks = p.k_new + o;
+                    vs = p.v_new + o;
+                }
+                cp_async16(st + cp.dst[i], ks);
+                cp_async16(st + (D / 64) * 2048 + cp.dst[i], vs);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) {
+                cp_async16(st + cp.dst[i], kb + cp.src[i]);
+                cp_async16(st + (D / 64) * 2048 + cp.dst[i], vb + cp.src[i]);
+            }
         }
     }
     c.b += NB;
@@ -420,8 +448,12 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
     const DecodeUnit first = p.units[unit];
     const CopyPattern<D> cpat(lane, Hkv * D);
     // the plan's tables are ready before the launch; the caller's data may be
-    // written by the kernel before this one (programmatic launch)
-    grid_dependency_wait();
+    // written by the kernel before this one (programmatic launch).  In a
+    // fused step that kernel is the cache scatter, started after everything
+    // before it had completed: the new keys come from k_new / v_new, no other
+    // data depends on it, and the wait moves to the end (so that what
+    // follows on the stream also follows the scatter).
+    if (p.wait_first) grid_dependency_wait();
 
     // Load cursor: this warp's next step to copy; S-1 steps run ahead.
     LoadCursor lc;
@@ -432,7 +464,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
         lc.r = st.row;
         lc.b = st.block;
         lc.done = st.row > run_end.row || (st.row == run_end.row && st.block >= run_end.block);
-        if (!lc.done) cursor_set_row(p, run_end, lc, st.seq, st.n_keys);
+        if (!lc.done) cursor_set_row(p, run_end, lc, st.seq, st.n_keys, st.token, st.n_new);
     }
 #pragma unroll
     for (int j = 0; j < S - 1; ++j) {
@@ -547,6 +579,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
         }
     });
     cp_async_wait<0>();  // nothing may still be landing when the warp exits
+    if (!p.wait_first) grid_dependency_wait();
 }
 
 // Merges every combine row, one warp per row: used when the decode kernel

@@ -29,6 +29,11 @@ struct DecodeParams {
     int max_blocks_per_seq;
     float scale_log2;
     int defer_merge;            // nonzero: split rows only write partials (merge_kernel follows)
+    // fused step: K/V of this step's tokens ([T][Hkv][D]), read instead of
+    // their cache slots (null: every key comes from the cache)
+    const __nv_bfloat16 *k_new;
+    const __nv_bfloat16 *v_new;
+    int wait_first;             // 0 only right behind the step's own scatter (see decode_kernel)
 };
 
 cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t *slots,

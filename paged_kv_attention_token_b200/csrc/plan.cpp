@@ -315,7 +315,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
             seg_row0[i] = (int)rows.size();
             for (int j = 0; j < L; ++j)
                 for (int g = 0; g < Hkv; ++g)
-                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, shared[i], {0, 0}});
+                    rows.push_back({h_cu[i] + j, i, n - L + j + 1, pa::kUnsplitRow, -1, shared[i], j + 1, 0});
         } else {
             const int nt = (int)cdiv(n, pa::kPrefillTileN);  // key tiles of the segment
             const int base = (int)stages.size();
@@ -433,9 +433,10 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
                 off = 0;
             }
             units[u] = {(int32_t)rr, (int32_t)off + (rr < R ? rows[rr].first_block : 0),
-                        rr < R ? rows[rr].seq : 0, rr < R ? rows[rr].n_keys : 0};
+                        rr < R ? rows[rr].seq : 0, rr < R ? rows[rr].n_keys : 0,
+                        rr < R ? rows[rr].token : 0, rr < R ? rows[rr].n_new : 0};
         }
-        units[P] = {(int32_t)R, 0, 0, 0};
+        units[P] = {(int32_t)R, 0, 0, 0, 0, 0};
     }
     // Pieces: a row is split if its blocks span more than one unit.
     std::vector<pa::CombineRow> combine;

@@ -35,7 +35,10 @@ struct DecodeRow {
     int32_t first_block;  // first block read here: > 0 when the row's leading
                           // blocks are a prefix shared with other rows,
                           // attended by the prefill kernel (cascade)
-    int32_t pad[2];
+    int32_t n_new;        // keys of the row written by this step: its segment's
+                          // new tokens up to its own (keys n_keys - n_new ..
+                          // n_keys - 1 are tokens token - n_new + 1 .. token)
+    int32_t pad;
 };
 
 // A decode warp's work: flat (row, block) range [start, next unit's start);
@@ -47,6 +50,8 @@ struct DecodeUnit {
     int32_t block;
     int32_t seq;     // rows[row].seq (0 for the end marker)
     int32_t n_keys;  // rows[row].n_keys (0 for the end marker)
+    int32_t token;   // rows[row].token (0 for the end marker)
+    int32_t n_new;   // rows[row].n_new (0 for the end marker)
 };
 
 // A row whose result is merged from partials: cut across several decode

@@ -195,6 +195,16 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(lib):
     assert lib.pa_attention_varlen(*args, plan.handle, ctypes.c_void_p(0x10010), 1 << 20, S) == pa.PA_ERR_WORKSPACE
     args_odd = [odd] + [fake] * 5 + [ctypes.c_float(0.125), fake, ctypes.byref(d)]
     assert lib.pa_attention_varlen(*args_odd, plan.handle, fake, 1 << 20, S) == pa.PA_ERR_ALIGN
+    # fused scatter + attention: its own pointers are checked before anything else
+    fused = lambda *a: lib.pa_reshape_and_attention(*a)
+    tail = [fake, fake, fake, fake, fake, fake, ctypes.c_float(0.125), fake, ctypes.byref(d), plan.handle, fake,
+            ctypes.c_size_t(1 << 20), S]
+    assert fused(None, fake, fake, fake, *tail[1:]) == pa.PA_ERR_NULL
+    assert fused(odd, fake, fake, fake, *tail[1:]) == pa.PA_ERR_ALIGN
+    assert fused(fake, fake, ctypes.c_void_p(0x10004), fake, *tail[1:]) == pa.PA_ERR_ALIGN  # slots: 8-byte aligned
+    assert fused(fake, fake, fake, fake, *tail[1:9], None, *tail[10:]) == pa.PA_ERR_NULL  # no plan
+    assert fused(S, S, S, S, S, S, S, S, S, ctypes.c_float(0.125), S, ctypes.byref(d0), plan.handle, S, 0, S) \
+        in (pa.PA_OK, pa.PA_ERR_PLAN)                                   # T = 0: nothing to check or queue
     # validate: scratch too small
     assert lib.pa_validate_inputs(fake, fake, fake, fake, ctypes.byref(d), fake, 8, S) == pa.PA_ERR_WORKSPACE
 
