@@ -259,6 +259,21 @@ def baseline_value(decode: bool, units: dict, sec: float) -> float:
 # the reference arm: the CPU oracle, as it stands
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The job's figure for a per-rank time: the max over ranks (each rank's
+    own value when there is one rank)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Seed of a rank's batch: every rank draws its own batch of the same shape."""
+    return W.WORKLOADS[workload][1] + 7919 * rank
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -313,8 +328,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pa.load_library()
 
-    fn, default_seed, _ = W.WORKLOADS[args.workload]
-    lay = W.layout(args.workload, seed=default_seed + 7919 * rank)
+    lay = W.layout(args.workload, seed=rank_seed(args.workload, rank))
     decode = is_decode_workload(lay)
     batch = W.make_batch(lay, device=dev)
     acct = step_bytes(lay)
@@ -379,10 +393,7 @@ def run_ours(args):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = max_total_ms / args.steps
 
     if decode:
@@ -485,10 +496,7 @@ def run_ours(args):
             e1.synchronize()
             if i >= args.warmup:
                 e_ms.append(e0.elapsed_time(e1))
-        te = torch.tensor([sum(e_ms)], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e_total = float(te.item())
+        e_total = max_over_ranks(sum(e_ms), dist, dev)
         e_val = (world * acct["total"] * args.steps / (e_total * 1e-3) / 1e9) if decode else \
             (world * lay.num_tokens * args.steps / (e_total * 1e-3))
         e2e = {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
