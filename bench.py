@@ -23,8 +23,9 @@ time is the max over ranks.
 
 The JSON line adds: roofline (dominant kernel, timed in the same run with
 CUDA events around it on its stream, in a second pass of K identical steps,
-since event records cost GPU time of their own), e2e (same metric through the public API with host buffers: H2D of
-the step's inputs and D2H of its output inside the timed region), the CPU
+since event records cost GPU time of their own), e2e (same metric through the public API with host buffers: the
+step's inputs, kept in one page-locked buffer, cross to the device in one copy; that copy, the plan build and
+the D2H of the output are inside the timed region), the CPU
 oracle as a reported baseline, SM clocks sampled during the timed region, and
 the number of library kernels launched.
 """
@@ -467,21 +468,31 @@ def run_ours(args):
     # e2e: public API with host buffers; H2D of the step's inputs, D2H of out
     e2e = None
     if not args.no_e2e:
-        host = {n: x.detach().cpu().pin_memory() for n, x in
-                (("q", batch.q), ("k", batch.k), ("v", batch.v), ("slots", slots),
-                 ("bt", bt), ("cu", cu), ("sl", sl))}
-        dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+        # the step's host inputs live in one page-locked buffer (each at a
+        # 256-byte offset) and cross to the device in one copy
+        srcs = (("q", batch.q), ("k", batch.k), ("v", batch.v), ("slots", slots),
+                ("bt", bt), ("cu", cu), ("sl", sl))
+        offs, nbytes = {}, 0
+        for n, x in srcs:
+            offs[n] = nbytes
+            nbytes += -(-x.numel() * x.element_size() // 256) * 256
+        h_stage = torch.zeros(nbytes, dtype=torch.uint8, pin_memory=True)
+        d_stage = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        dev_in = {}
+        for n, x in srcs:
+            nb = x.numel() * x.element_size()
+            h_stage[offs[n]:offs[n] + nb].copy_(x.detach().contiguous().view(-1).view(torch.uint8).cpu())
+            dev_in[n] = d_stage[offs[n]:offs[n] + nb].view(x.dtype).view(x.shape)
         out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         # inputs, plus the plan tables each step's build uploads
-        h2d = sum(x.numel() * x.element_size() for x in host.values()) + info["table_bytes"]
+        h2d = nbytes + info["table_bytes"]
         d2h = out_host.numel() * out_host.element_size()
         e_ms = []
         for i in range(args.warmup + args.steps):
             flush.fill_(2)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for n in host:
-                dev_in[n].copy_(host[n], non_blocking=True)
+            d_stage.copy_(h_stage, non_blocking=True)
             plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims, h_bt)
             if args.two_calls:
                 pa.reshape_and_cache(dev_in["k"], dev_in["v"], dev_in["slots"], kc, vc, stream=stream)

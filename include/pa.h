@@ -111,8 +111,9 @@ int pa_reshape_and_cache(const void *d_k, const void *d_v, const int64_t *d_slot
  * 128-query tiles for pairs of query heads sharing a kv head, for the
  * tensor-core prefill kernel and dealt to at most one CTA per SM.  The
  * resulting tables are uploaded to device memory the plan owns, on a stream
- * of the plan's own (an asynchronous copy from page-locked memory; the only
- * GPU work a build queues).
+ * of the plan's own (a copy from page-locked memory, the only GPU work a
+ * build queues); the call returns once they are on the device.  Build plans
+ * outside stream capture.
  *   h_cu_seqlens_q  host [S+1] int32
  *   h_seq_lens      host [S] int32
  *   h_block_tables  host [S][MB] int32 (the values the device array will
@@ -216,9 +217,12 @@ void pa_plan_destroy(pa_plan *plan);
  *                   in flight at once need two workspaces.
  * After a call that reported an error, rebuild the plan (its merge tickets
  * may be left taken) and reset the workspace's status word.
- * The call makes `stream` wait for the plan's upload (no wait once the host
- * has seen it complete), then queues its kernels; nothing is copied from the
- * host.  The decode kernel is launched with programmatic stream
+ * The call queues its kernels on `stream` and nothing else (the plan's tables
+ * are on the device since its build returned); nothing is copied from the
+ * host.  It may be captured into a CUDA graph (stream capture in any mode):
+ * a captured call does not record the plan's use, so a plan must not be
+ * rebuilt or destroyed while a graph replay that uses it may run, and
+ * replays that use one plan must not overlap.  The decode kernel is launched with programmatic stream
  * serialization: its blocks may start while the kernel queued before it on
  * `stream` is still running, read only the plan's tables until that kernel
  * has completed (griddepcontrol.wait), and then everything else.  Stream
@@ -237,7 +241,7 @@ int pa_attention_varlen(const void *d_q, const void *d_k_cache, const void *d_v_
  * non-NULL entry of trace->events (a cudaEvent_t created by the caller) is
  * recorded on `stream` at a fixed point of the call, so that the caller can
  * time every kernel on the stream it runs on:
- *   [0] before the wait for the plan's upload
+ *   [0] at the start of the call
  *   [1] before the split-KV decode kernel (which also merges split rows)
  *   [2] after the split-KV kernel      [3] = [2] (no separate combine kernel)
  *   [4] before the K/V staging and prefill kernels

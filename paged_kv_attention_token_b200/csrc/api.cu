@@ -176,19 +176,14 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const uint8_t *tb = static_cast<const uint8_t *>(plan->d_tables);
     if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
-    // the upload queued by the plan's build (usually long done: then no
-    // stream wait, which keeps the decode kernel's programmatic launch
-    // directly behind the caller's previous kernel)
-    {
-        cudaEvent_t up = static_cast<cudaEvent_t>(plan->upload_event);
-        const cudaError_t qs = cudaEventQuery(up);
-        if (qs == cudaErrorNotReady) {
-            if (cudaPeekAtLastError() == cudaErrorNotReady) cudaGetLastError();
-            if (cudaStreamWaitEvent(stream, up, 0) != cudaSuccess) return PA_ERR_CUDA;
-        } else if (qs != cudaSuccess) {
-            return PA_ERR_CUDA;
-        }
-    }
+    // The plan's tables are on the device since its build returned, so
+    // nothing sits between the caller's previous kernel and the decode
+    // kernel's programmatic launch.  Under stream capture (a CUDA graph) the
+    // plan-use event below is not recorded: a graph replay is not tracked by
+    // the plan, whose rebuild then must not overlap one.
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) return PA_ERR_CUDA;
+    const bool track_use = capture == cudaStreamCaptureStatusNone;
     const float scale_log2 = scale * kLog2e;
     DecodeParams p{};
     if (plan->num_units > 0) {
@@ -271,7 +266,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
             return PA_ERR_CUDA;
         if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
             return PA_ERR_CUDA;
-        if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
+            return PA_ERR_CUDA;
         return PA_OK;
     } else if (plan->cascade) {
         // shared-prefix partials first; the decode kernel merges them
@@ -281,7 +277,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         if (mark(trace, 5, stream) != cudaSuccess || mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
         if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
+            return PA_ERR_CUDA;
         return PA_OK;
     } else {
         if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
@@ -298,7 +295,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
     }
     if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;
     // the plan's next build waits for this
-    if (cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
+        return PA_ERR_CUDA;
     return PA_OK;
 }
 }  // namespace

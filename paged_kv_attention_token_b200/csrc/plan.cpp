@@ -217,7 +217,8 @@ bool create_sync_objects(pa_plan *p) {
 }
 
 // Copies the host image of the tables to the plan's device buffer on the
-// plan's stream (the caller has waited for the plan to be idle).
+// plan's stream and waits for the copy (the caller has waited for the plan
+// to be idle).
 bool upload_tables(pa_plan *p) {
     if (p->device < 0) return true;
     DeviceScope scope(p->device);
@@ -237,7 +238,10 @@ bool upload_tables(pa_plan *p) {
     }
     cudaStream_t s = static_cast<cudaStream_t>(p->upload_stream);
     if (cudaMemcpyAsync(p->d_tables, p->tables, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return false;
-    return cudaEventRecord(static_cast<cudaEvent_t>(p->upload_event), s) == cudaSuccess;
+    // the build returns with the tables on the device: attention calls then
+    // queue no wait for them (and can be captured into a CUDA graph)
+    if (cudaEventRecord(static_cast<cudaEvent_t>(p->upload_event), s) != cudaSuccess) return false;
+    return cudaEventSynchronize(static_cast<cudaEvent_t>(p->upload_event)) == cudaSuccess;
 }
 
 int check_dims(const pa_dims *d) {

@@ -95,3 +95,40 @@ def test_fused_consecutive_calls_and_side_stream(cuda_lib):
 def test_fused_without_host_tables(cuda_lib):
     # no shared-prefix detection: the prefix workload runs as plain decode
     check_against_two_calls(W.make_batch(W.layout("prefix_llama3_70b_b128"), device="cuda"), with_tables=False)
+
+
+@pytest.mark.parametrize("name", ["tiny_mixed", "decode_tinyllama_b64", "prefix_llama3_70b_b128",
+                                  "mixed_qwen25_1p5b_t8192"])
+def test_fused_step_captured_in_a_cuda_graph(cuda_lib, name):
+    # the step (scatter + attention, one call) captured once and replayed:
+    # decode only, shared prefix beside the suffix decode (merge kernel) and
+    # the side-by-side mixed step (a second stream joins the capture)
+    b = W.make_batch(W.layout(name), device="cuda")
+    kc_ref, vc_ref, ref, _ = run_step(b)
+    lay = b.layout
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    bt, cu, sl, slots = b.device_ints("cuda")
+    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, dims_for(lay), block_tables=lay.block_tables)
+    ws = pa.workspace_for(plan)
+    out = torch.empty_like(b.q)
+
+    def step():
+        pa.reshape_and_attention(b.k, b.v, slots, b.q, kc, vc, bt, cu, sl, b.scale, out, plan, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    out.fill_(float("nan"))
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert pa.workspace_status(ws) == 0
+    assert same_bits(kc, kc_ref) and same_bits(vc, vc_ref)
+    assert same_bits(out, ref)
+    del g
