@@ -26,8 +26,10 @@ CUDA events around it on its stream, in a second pass of K identical steps,
 since event records cost GPU time of their own), e2e (same metric through the public API with host buffers: the
 step's inputs, kept in one page-locked buffer, cross to the device in one copy; that copy, the plan build and
 the D2H of the output are inside the timed region), the CPU
-oracle as a reported baseline, SM clocks sampled during the timed region, and
-the number of library kernels launched.
+oracle as a reported baseline, SM clocks sampled during the timed region, the
+number of library kernels launched, and kv_transfer: pa_kv_export and
+pa_kv_import of every request's whole history, each timed alone (GB/s and the
+fraction of the measured HBM bandwidth).
 """
 from __future__ import annotations
 
@@ -513,6 +515,41 @@ def run_ours(args):
         e2e = {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_total / args.steps}
 
+    # KV export / import of every request's whole history (the local half of
+    # moving a request's KV between instances), each call timed alone with
+    # events after an L2 flush; algorithmic bytes: K and V of every token,
+    # read once and written once
+    kv_transfer = None
+    if not args.no_kv_transfer:
+        cu_t = torch.from_numpy(np.concatenate([[0], np.cumsum(lay.seq_lens)]).astype(np.int32)).to(dev)
+        n_tok = int(lay.seq_lens.sum())
+        k_buf = torch.empty((n_tok, lay.num_kv_heads, lay.head_dim), dtype=torch.bfloat16, device=dev)
+        v_buf = torch.empty_like(k_buf)
+        xfer_bytes = 2 * 2 * k_buf.numel() * k_buf.element_size()
+
+        def time_calls(fn):
+            ms = []
+            for i in range(args.warmup + args.steps):
+                flush.fill_(3)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                if i >= args.warmup:
+                    ms.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            return statistics.mean(a.elapsed_time(b) for a, b in ms)
+
+        exp_ms = time_calls(lambda: pa.kv_export(kc, vc, bt, cu_t, k_buf, v_buf, stream=stream))
+        # (importing the exported history back writes every slot the same value)
+        imp_ms = time_calls(lambda: pa.kv_import(k_buf, v_buf, bt, cu_t, kc, vc, stream=stream))
+        exp_gbs, imp_gbs = xfer_bytes / (exp_ms * 1e-3) / 1e9, xfer_bytes / (imp_ms * 1e-3) / 1e9
+        kv_transfer = {"tokens": n_tok, "bytes_per_call": xfer_bytes,
+                       "export": {"ms": exp_ms, "GB/s": exp_gbs, "frac": exp_gbs / peaks["hbm_gbs"]},
+                       "import": {"ms": imp_ms, "GB/s": imp_gbs, "frac": imp_gbs / peaks["hbm_gbs"]},
+                       "peak_kind": peak_kind}
+        del k_buf, v_buf
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host_batch = batch
@@ -544,6 +581,7 @@ def run_ours(args):
             "roofline": roofline,
             "roofline_decode": roofline_decode,
             "roofline_prefill": roofline_prefill,
+            "kv_transfer": kv_transfer,
             "step_roofline": step_roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -568,6 +606,7 @@ def main():
     ap.add_argument("--two-calls", action="store_true",
                     help="step through pa_reshape_and_cache + pa_attention_varlen instead of the fused call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kv-transfer", action="store_true", help="skip timing pa_kv_export / pa_kv_import")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -307,6 +307,39 @@ int pa_workspace_status(const void *d_workspace, void *stream, uint32_t *status)
 int pa_workspace_reset(void *d_workspace, const pa_plan *plan, void *stream);
 
 /*
+ * KV export and import ("vLLM 学习笔记 01" §2.5, prefill/decode
+ * disaggregation: a prefill instance produces a request's full KV cache and
+ * a connector carries it to a decode instance, which needs it in its own
+ * pool).  Export gathers the K/V of S requests from the paged cache into
+ * contiguous buffers; import writes such buffers into a pool through
+ * (possibly other) block tables.  Only the local device half: moving the
+ * buffers between instances is outside the library.
+ * Token p of request i (0 <= p < n_i = cu_tokens[i + 1] - cu_tokens[i]) is
+ * row cu_tokens[i] + p of the buffers and row p % 16 of cache block
+ * block_tables[i][p / 16].  Bit-for-bit copies; nothing else is touched.
+ *   d_k_cache, d_v_cache  device [NB][16][Hkv][D] bf16 (read by export,
+ *                         written by import)
+ *   d_block_tables        device [S][MB] int32
+ *   d_cu_tokens           device [S+1] int32: 0, non-decreasing, ends at N
+ *   d_k_out/d_v_out (export), d_k_in/d_v_in (import)  device [N][Hkv][D] bf16
+ *   dims                  host; num_tokens = N, num_seqs = S, num_kv_heads,
+ *                         head_dim, num_blocks, max_blocks_per_seq,
+ *                         block_size (16) are used
+ * Preconditions (not checked on the host): n_i <= MB * 16 and every table
+ * entry a request's tokens use is inside the pool; rows that break them are
+ * skipped without any access.  Import into slots another request also uses
+ * is undefined.  N == 0 queues nothing.
+ * Errors: PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_UNSUPPORTED,
+ * PA_ERR_CUDA.
+ */
+int pa_kv_export(const void *d_k_cache, const void *d_v_cache, const int32_t *d_block_tables,
+                 const int32_t *d_cu_tokens, void *d_k_out, void *d_v_out, const pa_dims *dims,
+                 void *stream);
+int pa_kv_import(const void *d_k_in, const void *d_v_in, const int32_t *d_block_tables,
+                 const int32_t *d_cu_tokens, void *d_k_cache, void *d_v_cache, const pa_dims *dims,
+                 void *stream);
+
+/*
  * Opt-in check of the data-dependent preconditions, on the device, then a
  * synchronize of `stream`: every slot_mapping entry is negative or inside the
  * pool; no two tokens share a slot; cu_seqlens_q starts at 0, is

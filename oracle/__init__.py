@@ -67,6 +67,10 @@ def _load():
             lib.oracle_attention_varlen.restype = ctypes.c_int
             lib.oracle_attention_varlen.argtypes = [
                 P, P, P, P, P, P, I32, I32, I32, I32, I64, I32, I32, D, P, I64, P, I32]
+            for name in ("oracle_kv_export", "oracle_kv_import"):
+                fn = getattr(lib, name)
+                fn.restype = ctypes.c_int
+                fn.argtypes = [P, P, I64, I32, I32, I32, P, I32, P, I32, P, P]
             lib.oracle_default_threads.restype = ctypes.c_int
             lib.oracle_default_threads.argtypes = []
             _lib = lib
@@ -156,3 +160,46 @@ def attention_varlen(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         S, Hq, Hkv, D, NB, MB, B, float(scale), _ptr(rows), n_rows, _ptr(out),
         int(threads)))
     return out
+
+
+def _kv_args(cache_k, cache_v, block_tables, cu_tokens, buf_k, buf_v):
+    NB, B, Hkv, D = cache_k.shape
+    if cache_v.shape != cache_k.shape or buf_k.shape != buf_v.shape or tuple(buf_k.shape[1:]) != (Hkv, D):
+        raise ValueError("shape mismatch")
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cu = np.ascontiguousarray(cu_tokens, dtype=np.int32)
+    S = bt.shape[0]
+    if bt.ndim != 2 or cu.shape != (S + 1,) or cu[-1] != buf_k.shape[0]:
+        raise ValueError("block_tables must be [S, MB] and cu_tokens [S+1] ending at N")
+    return NB, B, Hkv, D, bt, cu, S
+
+
+def kv_export(k_cache: np.ndarray, v_cache: np.ndarray, block_tables: np.ndarray,
+              cu_tokens: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """K/V of requests gathered from the caches into contiguous buffers.
+
+    Request i's token p (0 <= p < cu_tokens[i+1] - cu_tokens[i]) is read
+    from block block_tables[i][p // block_size], row p % block_size, and
+    becomes row cu_tokens[i] + p of the returned uint16 [N, Hkv, D] arrays.
+    """
+    k_cache, v_cache = _bits(k_cache), _bits(v_cache)
+    N = int(np.asarray(cu_tokens)[-1])
+    k_out = np.zeros((N,) + k_cache.shape[2:], dtype=np.uint16)
+    v_out = np.zeros_like(k_out)
+    NB, B, Hkv, D, bt, cu, S = _kv_args(k_cache, v_cache, block_tables, cu_tokens, k_out, v_out)
+    _check(_load().oracle_kv_export(_ptr(k_cache), _ptr(v_cache), NB, B, Hkv, D, _ptr(bt), bt.shape[1],
+                                    _ptr(cu), S, _ptr(k_out), _ptr(v_out)))
+    return k_out, v_out
+
+
+def kv_import(k_in: np.ndarray, v_in: np.ndarray, block_tables: np.ndarray, cu_tokens: np.ndarray,
+              k_cache: np.ndarray, v_cache: np.ndarray) -> None:
+    """Write contiguous K/V buffers into the caches (in place) through the
+    block tables: the inverse of kv_export for the slots the requests use."""
+    k_in, v_in = _bits(k_in), _bits(v_in)
+    if not (k_cache.flags.c_contiguous and v_cache.flags.c_contiguous):
+        raise ValueError("caches must be C-contiguous (they are written in place)")
+    _bits(k_cache), _bits(v_cache)
+    NB, B, Hkv, D, bt, cu, S = _kv_args(k_cache, v_cache, block_tables, cu_tokens, k_in, v_in)
+    _check(_load().oracle_kv_import(_ptr(k_in), _ptr(v_in), NB, B, Hkv, D, _ptr(bt), bt.shape[1],
+                                    _ptr(cu), S, _ptr(k_cache), _ptr(v_cache)))

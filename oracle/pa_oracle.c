@@ -17,6 +17,10 @@
  *  - same page, §1.4 and §2.1: a request tracks computed vs total tokens, so
  *    a segment's seq_len counts the tokens scheduled this step, and a
  *    prefill chunk reads the context cached by earlier chunks.
+ *  - same page, §2.5 (prefill/decode disaggregation): a prefill instance
+ *    produces a request's full KV cache and a connector moves it to a decode
+ *    instance; kv_export / kv_import state the local half, a request's K/V
+ *    between its blocks and one contiguous buffer.
  *  - "Inside vLLM: Anatomy of a High-Throughput LLM Inference System"
  *    (Chinese translation), section "LLM 引擎构造函数" (engine constructor),
  *    KV cache manager paragraph: one block of a standard (non-MLA) layer holds
@@ -97,6 +101,73 @@ int oracle_reshape_and_cache(const uint16_t *k, const uint16_t *v,
         }
     }
     return ORACLE_OK;
+}
+
+/*
+ * kv_export / kv_import: request i (0 <= i < num_seqs) owns buffer rows
+ * cu_tokens[i] .. cu_tokens[i + 1] - 1; its token p is row p of that range
+ * and row p % block_size of cache block block_tables[i][p / block_size].
+ * Export copies every such token's K and V (all kv heads) from the caches to
+ * the buffers, import the other way; bitwise.  Nothing else is touched.
+ */
+static int kv_transfer(int do_export, uint16_t *k_cache, uint16_t *v_cache, int64_t num_blocks,
+                       int block_size, int num_kv_heads, int head_dim, const int32_t *block_tables,
+                       int max_blocks_per_seq, const int32_t *cu_tokens, int num_seqs,
+                       uint16_t *k_buf, uint16_t *v_buf)
+{
+    if (num_seqs < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0 ||
+        max_blocks_per_seq < 0)
+        return ORACLE_ERR_ARG;
+    if (num_seqs == 0)
+        return ORACLE_OK;
+    if (!k_cache || !v_cache || !block_tables || !cu_tokens || !k_buf || !v_buf)
+        return ORACLE_ERR_ARG;
+    if (cu_tokens[0] != 0)
+        return ORACLE_ERR_SEGMENT;
+    for (int i = 0; i < num_seqs; ++i) {
+        int n = cu_tokens[i + 1] - cu_tokens[i];
+        if (n < 0 || (int64_t)n > (int64_t)max_blocks_per_seq * block_size)
+            return ORACLE_ERR_SEGMENT;
+        for (int b = 0; b * block_size < n; ++b) {
+            int32_t id = block_tables[(int64_t)i * max_blocks_per_seq + b];
+            if (id < 0 || id >= num_blocks)
+                return ORACLE_ERR_BLOCK;
+        }
+    }
+    const int64_t token_elems = (int64_t)num_kv_heads * head_dim;
+    for (int i = 0; i < num_seqs; ++i) {
+        for (int p = 0; p < cu_tokens[i + 1] - cu_tokens[i]; ++p) {
+            int64_t block = block_tables[(int64_t)i * max_blocks_per_seq + p / block_size];
+            int64_t cache_row = block * block_size + p % block_size;
+            int64_t buf_row = (int64_t)cu_tokens[i] + p;
+            for (int64_t e = 0; e < token_elems; ++e) {
+                if (do_export) {
+                    k_buf[buf_row * token_elems + e] = k_cache[cache_row * token_elems + e];
+                    v_buf[buf_row * token_elems + e] = v_cache[cache_row * token_elems + e];
+                } else {
+                    k_cache[cache_row * token_elems + e] = k_buf[buf_row * token_elems + e];
+                    v_cache[cache_row * token_elems + e] = v_buf[buf_row * token_elems + e];
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_kv_export(const uint16_t *k_cache, const uint16_t *v_cache, int64_t num_blocks, int block_size,
+                     int num_kv_heads, int head_dim, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *cu_tokens, int num_seqs, uint16_t *k_out, uint16_t *v_out)
+{
+    return kv_transfer(1, (uint16_t *)k_cache, (uint16_t *)v_cache, num_blocks, block_size, num_kv_heads,
+                       head_dim, block_tables, max_blocks_per_seq, cu_tokens, num_seqs, k_out, v_out);
+}
+
+int oracle_kv_import(const uint16_t *k_in, const uint16_t *v_in, int64_t num_blocks, int block_size,
+                     int num_kv_heads, int head_dim, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *cu_tokens, int num_seqs, uint16_t *k_cache, uint16_t *v_cache)
+{
+    return kv_transfer(0, k_cache, v_cache, num_blocks, block_size, num_kv_heads, head_dim, block_tables,
+                       max_blocks_per_seq, cu_tokens, num_seqs, (uint16_t *)k_in, (uint16_t *)v_in);
 }
 
 typedef struct {

@@ -94,6 +94,8 @@ def load_library():
             "pa_attention_varlen_ex": (I, [P, P, P, P, P, P, F, P, DP, P, P, SZ, P, P]),
             "pa_attention_varlen_noalloc": (I, [P, P, P, P, P, P, F, P, DP, P, P]),
             "pa_reshape_and_attention": (I, [P, P, P, P, P, P, P, P, P, F, P, DP, P, P, SZ, P]),
+            "pa_kv_export": (I, [P, P, P, P, P, P, DP, P]),
+            "pa_kv_import": (I, [P, P, P, P, P, P, DP, P]),
             "pa_noalloc_scratch_bytes": (SZ, []),
             "pa_workspace_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "pa_workspace_reset": (I, [P, P, P]),
@@ -331,6 +333,38 @@ def reshape_and_attention(k, v, slot_mapping, q, k_cache, v_cache, block_tables,
         ctypes.byref(d), plan.handle, _dev_ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel()),
         _stream_ptr(stream)), "pa_reshape_and_attention")
     return out
+
+
+def _kv_transfer(name, src_k, src_v, dst_k, dst_v, cache, buf, block_tables, cu_tokens, stream):
+    lib = load_library()
+    if buf.dim() != 3 or cache.dim() != 4 or tuple(cache.shape[2:]) != tuple(buf.shape[1:]):
+        raise PaError(PA_ERR_SHAPE, f"{name}: cache [NB,16,Hkv,D] and buffers [N,Hkv,D] disagree")
+    if block_tables.dim() != 2 or tuple(cu_tokens.shape) != (block_tables.shape[0] + 1,):
+        raise PaError(PA_ERR_SHAPE, f"{name}: block_tables [S,MB] and cu_tokens [S+1]")
+    N, Hkv, D = buf.shape
+    d = Dims(N, block_tables.shape[0], Hkv, Hkv, D, cache.shape[0], block_tables.shape[1], cache.shape[1])
+    bf = torch.bfloat16
+    _check(getattr(lib, name)(_dev_ptr(src_k, "src_k", bf), _dev_ptr(src_v, "src_v", bf),
+                              _dev_ptr(block_tables, "block_tables", torch.int32),
+                              _dev_ptr(cu_tokens, "cu_tokens", torch.int32),
+                              _dev_ptr(dst_k, "dst_k", bf), _dev_ptr(dst_v, "dst_v", bf),
+                              ctypes.byref(d), _stream_ptr(stream)), name)
+
+
+def kv_export(k_cache, v_cache, block_tables, cu_tokens, k_out, v_out, stream=None) -> None:
+    """Gather requests' K/V from the paged caches into contiguous [N,Hkv,D]
+    buffers (pa_kv_export)."""
+    if k_out.shape != v_out.shape or k_cache.shape != v_cache.shape:
+        raise PaError(PA_ERR_SHAPE, "pa_kv_export: k/v shapes differ")
+    _kv_transfer("pa_kv_export", k_cache, v_cache, k_out, v_out, k_cache, k_out, block_tables, cu_tokens, stream)
+
+
+def kv_import(k_in, v_in, block_tables, cu_tokens, k_cache, v_cache, stream=None) -> None:
+    """Write contiguous [N,Hkv,D] K/V buffers into the paged caches through
+    the block tables (pa_kv_import)."""
+    if k_in.shape != v_in.shape or k_cache.shape != v_cache.shape:
+        raise PaError(PA_ERR_SHAPE, "pa_kv_import: k/v shapes differ")
+    _kv_transfer("pa_kv_import", k_in, v_in, k_cache, v_cache, k_cache, k_in, block_tables, cu_tokens, stream)
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:

@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "transfer.h"
 
 namespace pa {
 
@@ -334,6 +335,41 @@ extern "C" int pa_reshape_and_attention(const void *k, const void *v, const int6
         return PA_ERR_CUDA;
     return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, d, plan,
                            workspace, stream, nullptr, k, v);
+}
+
+namespace {
+int kv_transfer(bool do_export, const void *src_k, const void *src_v, void *dst_k, void *dst_v,
+                const int32_t *block_tables, const int32_t *cu_tokens, const pa_dims *dims, void *stream) {
+    if (!dims) return PA_ERR_NULL;
+    const pa_dims &d = *dims;
+    if (d.num_tokens < 0 || d.num_seqs < 0 || d.num_kv_heads <= 0 || d.head_dim <= 0 || d.num_blocks <= 0 ||
+        d.max_blocks_per_seq < 0 || d.block_size <= 0)
+        return PA_ERR_SHAPE;
+    if (d.block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (d.head_dim != 64 && d.head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (d.num_tokens == 0 || d.num_seqs == 0) return d.num_tokens == 0 ? PA_OK : PA_ERR_SHAPE;
+    if (!src_k || !src_v || !dst_k || !dst_v || !block_tables || !cu_tokens) return PA_ERR_NULL;
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(cu_tokens) & 3u))
+        return PA_ERR_ALIGN;
+    const cudaError_t e = launch_kv_transfer(do_export, src_k, src_v, dst_k, dst_v, block_tables, cu_tokens,
+                                             d.num_seqs, d.max_blocks_per_seq, d.num_blocks, d.num_tokens,
+                                             d.num_kv_heads * d.head_dim, current_sm_count(),
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" int pa_kv_export(const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                            const int32_t *cu_tokens, void *k_out, void *v_out, const pa_dims *dims,
+                            void *stream) {
+    return kv_transfer(true, k_cache, v_cache, k_out, v_out, block_tables, cu_tokens, dims, stream);
+}
+
+extern "C" int pa_kv_import(const void *k_in, const void *v_in, const int32_t *block_tables,
+                            const int32_t *cu_tokens, void *k_cache, void *v_cache, const pa_dims *dims,
+                            void *stream) {
+    return kv_transfer(false, k_in, v_in, k_cache, v_cache, block_tables, cu_tokens, dims, stream);
 }
 
 extern "C" int pa_workspace_reset(void *workspace, const pa_plan *plan, void *stream_) {

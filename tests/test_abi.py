@@ -205,6 +205,20 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(lib):
     assert fused(fake, fake, fake, fake, *tail[1:9], None, *tail[10:]) == pa.PA_ERR_NULL  # no plan
     assert fused(S, S, S, S, S, S, S, S, S, ctypes.c_float(0.125), S, ctypes.byref(d0), plan.handle, S, 0, S) \
         in (pa.PA_OK, pa.PA_ERR_PLAN)                                   # T = 0: nothing to check or queue
+    # KV export / import
+    for name in ("pa_kv_export", "pa_kv_import"):
+        fn = getattr(lib, name)
+        dk = dims_for(lay)
+        assert fn(S, S, S, S, S, S, None, S) == pa.PA_ERR_NULL
+        assert fn(None, fake, fake, fake, fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_NULL
+        assert fn(odd, fake, fake, fake, fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_ALIGN
+        assert fn(fake, fake, fake, ctypes.c_void_p(0x10002), fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_ALIGN
+        dk.head_dim = 96
+        assert fn(fake, fake, fake, fake, fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_UNSUPPORTED
+        dk = dims_for(lay); dk.num_tokens = 0
+        assert fn(S, S, S, S, S, S, ctypes.byref(dk), S) == pa.PA_OK          # nothing to move
+        dk = dims_for(lay); dk.num_seqs = 0
+        assert fn(fake, fake, fake, fake, fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_SHAPE  # rows, no requests
     # validate: scratch too small
     assert lib.pa_validate_inputs(fake, fake, fake, fake, ctypes.byref(d), fake, 8, S) == pa.PA_ERR_WORKSPACE
 

@@ -392,3 +392,84 @@ def test_tolerance_catches_a_wrong_kv_head_mapping():
     q2 = q[:, [0, 2, 1, 3]]
     bad = O.attention_varlen(q2, kc, vc, lay.block_tables, lay.cu_seqlens_q, lay.seq_lens, b.scale)[:, [0, 2, 1, 3]]
     assert not within(bad.astype(np.float32), good)
+
+
+# --------------------------------------------------------------------------
+# KV export / import ("vLLM 学习笔记 01" §2.5: a request's KV cache moved
+# between instances; the local half is a gather to / scatter from a
+# contiguous buffer through the block table)
+# --------------------------------------------------------------------------
+
+def _cu_tokens(seq_lens):
+    return np.concatenate([[0], np.cumsum(seq_lens)]).astype(np.int32)
+
+
+def test_kv_export_returns_each_requests_dense_history():
+    # the pool is built block by block from dense per-request K/V (numpy
+    # slicing); export must give those dense arrays back, concatenated
+    seq_lens = [33, 1, 16, 70, 0, 17]
+    lay, _, Kd, Vd, kc, vc = dense_problem([1, 1, 1, 1, 0, 1], seq_lens, 4, 2, 64, seed=21)
+    k_out, v_out = O.kv_export(kc, vc, lay.block_tables, _cu_tokens(seq_lens))
+    assert np.array_equal(k_out, bits(np.concatenate(Kd)))
+    assert np.array_equal(v_out, bits(np.concatenate(Vd)))
+
+
+def test_kv_export_after_scatter_returns_the_written_tokens():
+    # a step's new tokens, written by the scatter, come back from export at
+    # their positions n - L .. n - 1
+    lay = W.custom_layout([1, 5, 17, 3], [33, 5, 40, 16], 6, 3, 64, 40, seed=5)
+    b = W.make_batch(lay)
+    kc, vc = scattered(b)
+    k_out, v_out = O.kv_export(kc, vc, lay.block_tables, _cu_tokens(lay.seq_lens))
+    k, v = W.bf16_bits(b.k), W.bf16_bits(b.v)
+    cu_t = _cu_tokens(lay.seq_lens)
+    for i in range(lay.num_seqs):
+        n, L = int(lay.seq_lens[i]), int(lay.q_lens[i])
+        rows = np.arange(cu_t[i] + n - L, cu_t[i] + n)
+        tok = np.arange(lay.cu_seqlens_q[i], lay.cu_seqlens_q[i + 1])
+        assert np.array_equal(k_out[rows], k[tok]) and np.array_equal(v_out[rows], v[tok])
+
+
+def test_kv_import_into_another_pool_gives_the_same_attention():
+    # export from one pool, import into an empty pool with other block ids:
+    # attention over the new pool is bit-identical, and only the slots the
+    # requests use are written
+    lay = W.custom_layout([1, 6, 1, 2], [39, 23, 64, 100], 8, 2, 64, 40, seed=13)
+    b = W.make_batch(lay)
+    kc, vc = scattered(b)
+    cu_t = _cu_tokens(lay.seq_lens)
+    k_buf, v_buf = O.kv_export(kc, vc, lay.block_tables, cu_t)
+    NB2 = lay.num_blocks + 25
+    used = int(sum(-(-int(n) // 16) for n in lay.seq_lens))
+    ids = np.random.default_rng(3).permutation(NB2)[:used].astype(np.int32)
+    bt2 = np.zeros_like(lay.block_tables)
+    o = 0
+    for i, n in enumerate(lay.seq_lens):
+        nb = -(-int(n) // 16)
+        bt2[i, :nb] = ids[o:o + nb]
+        o += nb
+    kc2 = np.full((NB2,) + kc.shape[1:], 0x7fc1, dtype=np.uint16)   # a NaN payload
+    vc2 = kc2.copy()
+    O.kv_import(k_buf, v_buf, bt2, cu_t, kc2, vc2)
+    q = W.bf16_bits(b.q)
+    out = O.attention_varlen(q, kc, vc, lay.block_tables, lay.cu_seqlens_q, lay.seq_lens, b.scale)
+    out2 = O.attention_varlen(q, kc2, vc2, bt2, lay.cu_seqlens_q, lay.seq_lens, b.scale)
+    assert not np.isnan(out).any() and np.array_equal(out, out2)
+    written = np.zeros(kc2.shape[:2], bool)
+    for i, n in enumerate(lay.seq_lens):
+        for p in range(int(n)):
+            written[bt2[i, p // 16], p % 16] = True
+    assert np.all(kc2[~written] == 0x7fc1) and np.all(vc2[~written] == 0x7fc1)
+    # and the round trip returns the buffers
+    k3, v3 = O.kv_export(kc2, vc2, bt2, cu_t)
+    assert np.array_equal(k3, k_buf) and np.array_equal(v3, v_buf)
+
+
+def test_kv_transfer_rejects_blocks_outside_the_pool_and_overlong_requests():
+    lay, _, _, _, kc, vc = dense_problem([1, 1], [20, 5], 4, 2, 64, seed=2)
+    bt = lay.block_tables.copy()
+    bt[0, 1] = lay.num_blocks
+    with pytest.raises(O.OracleError):
+        O.kv_export(kc, vc, bt, _cu_tokens([20, 5]))
+    with pytest.raises(O.OracleError):
+        O.kv_export(kc, vc, lay.block_tables, _cu_tokens([20, 16 * lay.max_blocks_per_seq + 1]))
