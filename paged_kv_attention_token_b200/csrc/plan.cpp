@@ -311,6 +311,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
             group_of[i] = (int)k;
         }
     std::vector<int> group_splits(groups.size(), 0);
+    rows.reserve((size_t)d.num_tokens * Hkv);
     for (int i = 0; i < d.num_seqs; ++i) {
         const int L = h_cu[i + 1] - h_cu[i];
         const int n = h_seq[i];
@@ -427,8 +428,18 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     std::vector<int64_t> ustart(P + 1);
     {
         int64_t r = 0;
+        // f = floor(total_cost * u / P), stepped without a division per unit
+        const int64_t step = P ? total_cost / P : 0, rem = P ? total_cost % P : 0;
+        int64_t f = 0, carry = 0;
         for (int64_t u = 0; u <= P; ++u) {
-            const int64_t f = P ? total_cost * u / P : 0;
+            if (u > 0) {
+                f += step;
+                carry += rem;
+                if (carry >= P) {
+                    ++f;
+                    carry -= P;
+                }
+            }
             ustart[u] = f;
             while (r < R && prefix[r + 1] <= f) ++r;  // row whose cost span holds f
             int64_t rr = r, off = r < R ? f - prefix[r] : 0;
@@ -444,6 +455,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     }
     // Pieces: a row is split if its blocks span more than one unit.
     std::vector<pa::CombineRow> combine;
+    combine.reserve((size_t)R);
     int32_t piece_base = 0;
     {
         int64_t u = 0;
