@@ -223,8 +223,9 @@ void pa_plan_destroy(pa_plan *plan);
  * a captured call does not record the plan's use, so a plan must not be
  * rebuilt or destroyed while a graph replay that uses it may run, and
  * replays that use one plan must not overlap; the first call on a device
- * (which sets kernel attributes) belongs before the capture, as a warm-up.  The decode kernel is launched with programmatic stream
- * serialization: its blocks may start while the kernel queued before it on
+ * (which sets kernel attributes) belongs before the capture, as a warm-up.
+ * The decode kernel is launched with programmatic stream serialization: its
+ * blocks may start while the kernel queued before it on
  * `stream` is still running, read only the plan's tables until that kernel
  * has completed (griddepcontrol.wait), and then everything else.  Stream
  * order is therefore kept for all caller data.
