@@ -311,7 +311,14 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
             group_of[i] = (int)k;
         }
     std::vector<int> group_splits(groups.size(), 0);
-    rows.reserve((size_t)d.num_tokens * Hkv);
+    {
+        size_t decode_tokens = 0;  // rows are made for the decode segments only
+        for (int i = 0; i < d.num_seqs; ++i) {
+            const int L = h_cu[i + 1] - h_cu[i];
+            if (L > 0 && (L <= pa::kDecodeMaxQLen || !pa::prefill_kernel_available())) decode_tokens += (size_t)L;
+        }
+        rows.reserve(decode_tokens * Hkv);
+    }
     for (int i = 0; i < d.num_seqs; ++i) {
         const int L = h_cu[i + 1] - h_cu[i];
         const int n = h_seq[i];
