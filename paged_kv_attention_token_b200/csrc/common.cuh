@@ -141,28 +141,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-// 4-D tiled TMA load (no multicast) into shared memory, completion counted
-// in bytes on `bar`.  `map` is the generic address of a __grid_constant__
-// CUtensorMap kernel parameter.  c0 (the innermost coordinate) must be a
-// multiple of 8 elements of bf16 (16 bytes).
-__device__ __forceinline__ void tma_load_4d(void *dst, const void *map, uint64_t *bar, int c0, int c1,
-                                            int c2, int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *map, uint64_t *bar, int c0, int c1, int c2,
-                                            int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Bulk copy (no tensor map, no multicast) of `bytes` contiguous bytes from
 // global to shared memory, completion counted on `bar`; both addresses
 // 16-byte aligned, bytes a multiple of 16.
@@ -172,7 +150,10 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
-// 3-D tiled TMA load (no multicast), as tma_load_4d.
+// 3-D tiled TMA load (no multicast) into shared memory, completion counted
+// in bytes on `bar`.  `map` is the generic address of a __grid_constant__
+// CUtensorMap kernel parameter; c0 (the innermost coordinate) must be a
+// multiple of 8 bf16 elements (16 bytes).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, uint64_t *bar, int c0, int c1, int c2) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
@@ -191,21 +172,12 @@ __device__ __forceinline__ void warpgroup_reg_alloc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-__device__ __forceinline__ void prefetch_tensormap(const void *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
 __device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
     uint4 r;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                  : "r"(addr));
     return r;
-}
-
-// Named barrier over `count` threads (a subset of the CTA).
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Byte address of 16-byte chunk `chunk` (0..7) of row `row` in a tile of
@@ -234,10 +206,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // D[tmem] (+)= A[smem] * B[smem], bf16 inputs, fp32 accumulators; issued by one thread.
 __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {

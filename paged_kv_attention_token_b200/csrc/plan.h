@@ -142,11 +142,11 @@ struct pa_plan {
     pa::TableLayout tl;
     pa::WorkspaceLayout ws;
     // Host image of the tables (page-locked when the plan has a device) and
-    // its device copy.  A build uploads the image on the plan's own stream
-    // and records upload_event; every attention call makes its stream wait
-    // for upload_event and records use_event after its last kernel.  A
-    // rebuild or destroy first waits for both, so that neither buffer
-    // changes under a queued copy or a running kernel.
+    // its device copy.  A build uploads the image on the plan's own stream,
+    // records upload_event and waits for it; every attention call outside
+    // stream capture records use_event after its last kernel.  A rebuild or
+    // destroy first waits for both, so that neither buffer changes under a
+    // queued copy or a running kernel.
     uint8_t *tables = nullptr;
     size_t tables_capacity = 0;
     bool tables_pinned = false;
