@@ -205,9 +205,8 @@ class Plan:
         if self._bt is not None and (self._bt.ndim != 2 or self._bt.shape[0] != self.dims.num_seqs
                                      or self._bt.shape[1] != self.dims.max_blocks_per_seq):
             raise ValueError(f"block_tables must be [{self.dims.num_seqs}][{self.dims.max_blocks_per_seq}]")
-        bt_ptr = None if self._bt is None else self._bt.ctypes.data_as(ctypes.c_void_p)
-        _check(self._lib.pa_plan_build(self._cu.ctypes.data_as(ctypes.c_void_p),
-                                       self._sl.ctypes.data_as(ctypes.c_void_p), bt_ptr,
+        bt_ptr = None if self._bt is None else self._bt.ctypes.data
+        _check(self._lib.pa_plan_build(self._cu.ctypes.data, self._sl.ctypes.data, bt_ptr,
                                        ctypes.byref(self.dims), self.device, ctypes.byref(self._h)),
                "pa_plan_build")
         return self
