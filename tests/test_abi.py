@@ -241,3 +241,43 @@ def test_attention_launch_count(lib, name):
     if name == "prefix_llama3_70b_b128":
         # 128 decodes on a 4096-token prefix: prefix tiles beside the suffix decode
         assert info["num_prefix_groups"] == 1 and info["attention_launches"] == 4
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_plan_invariants_on_random_batches(lib, seed):
+    # random mixes of decodes, speculative-decode rows, chunks and fresh
+    # prompts, head counts and head_dims: the planner's accounting holds
+    rng = np.random.default_rng(9000 + seed)
+    S = int(rng.integers(1, 200))
+    seq = rng.integers(1, 6000, S)
+    kind = rng.integers(0, 4, S)
+    q = np.where(kind == 0, 1, np.where(kind == 1, rng.integers(2, 17, S),
+                                        np.where(kind == 2, rng.integers(17, 700, S), seq)))
+    q = np.minimum(q, seq).astype(np.int32)
+    seq = seq.astype(np.int32)
+    cu = np.concatenate([[0], np.cumsum(q)]).astype(np.int32)
+    Hkv = int(2 ** rng.integers(0, 4))
+    G = int(rng.integers(1, 17))
+    D = int(rng.choice([64, 128]))
+    MB = int(-(-seq.max() // 16))
+    d = pa.Dims(int(cu[-1]), S, Hkv * G, Hkv, D, 1 << 20, MB, 16)
+    info = pa.Plan(cu, seq, d, device=-1).info()
+    dec = q <= 16
+    rows = int(q[dec].sum()) * Hkv
+    assert info["num_decode_rows"] == rows
+    blocks = sum(-(-(int(n) - int(L) + j + 1) // 16) for L, n in zip(q[dec], seq[dec]) for j in range(int(L)))
+    assert info["decode_kv_blocks"] == blocks * Hkv
+    warps_per_sm = 12 if D == 64 else 8
+    assert (info["num_decode_units"] == 0) == (blocks == 0)
+    assert info["num_decode_units"] <= 148 * warps_per_sm
+    assert info["num_partials"] >= 2 * info["num_combine_rows"]
+    assert info["num_partials"] <= info["num_combine_rows"] + info["num_decode_units"] * 2
+    # prefill: one tile per (128-query chunk, kv head, query-head pair)
+    tiles = sum(-(-int(L) // 128) for L in q[~dec]) * Hkv * (-(-G // 2))
+    assert info["num_prefill_tiles"] == tiles
+    pairs = sum(int(n) - int(L) + j + 1 for L, n in zip(q[~dec], seq[~dec]) for j in range(int(L)))
+    assert info["prefill_causal_pairs"] == pairs
+    assert info["num_staged_kv_tiles"] == sum(-(-int(n) // 128) for n in seq[~dec]) * Hkv
+    base = (info["num_decode_units"] > 0) + 2 * (info["num_prefill_tiles"] > 0)
+    assert info["attention_launches"] == base            # no shared prefixes without host tables
+    assert info["workspace_bytes"] >= 256 + info["num_partials"] * G * D * 4
