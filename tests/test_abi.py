@@ -281,3 +281,52 @@ def test_plan_invariants_on_random_batches(lib, seed):
     base = (info["num_decode_units"] > 0) + 2 * (info["num_prefill_tiles"] > 0)
     assert info["attention_launches"] == base            # no shared prefixes without host tables
     assert info["workspace_bytes"] >= 256 + info["num_partials"] * G * D * 4
+
+
+def test_shared_prefix_detection_on_constructed_tables(lib):
+    # runs of >= 4 consecutive single-token segments whose tables agree on
+    # >= 16 leading blocks (blocks wholly before each query's own key) form
+    # a group; the decode rows then read only the blocks after the prefix
+    rng = np.random.default_rng(77)
+    pool = rng.permutation(100000).astype(np.int32)
+    nxt = [0]
+
+    def fresh(n):
+        ids = pool[nxt[0]:nxt[0] + n]
+        nxt[0] += n
+        return list(ids)
+
+    segs = []   # (q_len, seq_len, table, shared blocks expected)
+    pa_ = fresh(20)
+    for s in (5, 40, 77, 3, 16, 90):           # 6 decodes on a 20-block prefix
+        n = 20 * 16 + s
+        segs.append((1, n, pa_ + fresh(-(-n // 16) - 20), 20))
+    pb = fresh(18)
+    for s in (7, 9, 11):                        # only 3: no group
+        n = 18 * 16 + s
+        segs.append((1, n, pb + fresh(-(-n // 16) - 18), 0))
+    segs.append((300, 900, fresh(-(-900 // 16)), 0))   # a prefill segment breaks runs
+    pc = fresh(16)
+    for s in (1, 2, 30, 60, 17):                # 5 decodes on a 16-block prefix
+        n = 16 * 16 + s
+        segs.append((1, n, pc + fresh(-(-n // 16) - 16), 16))
+    q = np.array([a for a, _, _, _ in segs], np.int32)
+    sl = np.array([b for _, b, _, _ in segs], np.int32)
+    MB = max(len(t) for _, _, t, _ in segs)
+    bt = np.zeros((len(segs), MB), np.int32)
+    for i, (_, _, t, _) in enumerate(segs):
+        bt[i, :len(t)] = t
+    cu = np.concatenate([[0], np.cumsum(q)]).astype(np.int32)
+    Hkv, G, D = 2, 4, 128
+    d = pa.Dims(int(cu[-1]), len(segs), Hkv * G, Hkv, D, 100000, MB, 16)
+    with_tables = pa.Plan(cu, sl, d, device=-1, block_tables=bt).info()
+    without = pa.Plan(cu, sl, d, device=-1).info()
+    assert with_tables["num_prefix_groups"] == 2 and without["num_prefix_groups"] == 0
+    dec = [(n, sh) for L, n, _, sh in segs if L == 1]
+    assert without["decode_kv_blocks"] == sum(-(-n // 16) for n, _ in dec) * Hkv
+    assert with_tables["decode_kv_blocks"] == sum(-(-n // 16) - sh for n, sh in dec) * Hkv
+    # the prefix tiles join the prefill segment's tiles and pairs
+    assert with_tables["num_prefill_tiles"] > without["num_prefill_tiles"]
+    extra_pairs = (6 * 20 + 5 * 16) * 16
+    assert with_tables["prefill_causal_pairs"] == without["prefill_causal_pairs"] + extra_pairs
+    assert with_tables["attention_launches"] in (3, 4)
