@@ -9,8 +9,9 @@ one call (pa_reshape_and_attention: the scatter kernel, the split-KV decode
 kernel + combine, and the tensor-core prefill kernel when the batch holds long
 segments; with --two-calls, pa_reshape_and_cache then pa_attention_varlen).  Inputs are
 seeded and synthetic with the shapes of the named workload (model names give
-attention shapes only; no weights).  Default workload: 64 decodes with the
-TinyLlama-1.1B attention shape.
+attention shapes only; no weights).  Default workload: the 8192-token mixed
+chunked-prefill step with the Qwen2.5-1.5B attention shape (1152 decodes, a
+2048-token chunk on 6144 cached tokens, fresh prompts of 1024/1536/2432).
 
 Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier and
 torch.cuda.synchronize() on both sides.  L2 is flushed (a 1 GiB write)
@@ -23,13 +24,18 @@ time is the max over ranks.
 
 The JSON line adds: roofline (dominant kernel, timed in the same run with
 CUDA events around it on its stream, in a second pass of K identical steps,
-since event records cost GPU time of their own), e2e (same metric through the public API with host buffers: the
-step's inputs, kept in one page-locked buffer, cross to the device in one copy; that copy, the plan build and
-the D2H of the output are inside the timed region), the CPU
-oracle as a reported baseline, SM clocks sampled during the timed region, the
-number of library kernels launched, and kv_transfer: pa_kv_export and
-pa_kv_import of every request's whole history, each timed alone (GB/s and the
-fraction of the measured HBM bandwidth).
+since event records cost GPU time of their own), the scatter kernel's own
+roofline (back-to-back launches on distinct inputs and slots, after an L2
+flush), e2e (same metric through the public API with host buffers: after a
+flush and a synchronize, the host clock runs from before the step's plan
+build through the copy of its inputs, kept in one page-locked buffer, to the
+device, the step itself and the copy of its output back, until that copy has
+landed; the step's e2e time is the larger of that host interval and the
+events around the same work), the host cost of a plan build on an idle
+plan, the CPU oracle as a reported baseline, SM clocks sampled during the
+timed region, the number of library kernels launched, and kv_transfer:
+pa_kv_export and pa_kv_import of every request's whole history, each timed
+alone (GB/s and the fraction of the measured HBM bandwidth).
 """
 from __future__ import annotations
 
@@ -54,7 +60,7 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "paged-attn decode KV GB/s (% of HBM peak); mixed-batch attn tokens/s, % roofline"
-DEFAULT_WORKLOAD = "decode_tinyllama_b64"
+DEFAULT_WORKLOAD = "mixed_qwen25_1p5b_t8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 1 << 30
 
@@ -78,14 +84,15 @@ def step_bytes(lay: W.Layout) -> dict:
 
 def decode_prefill_split(lay: W.Layout, info: dict):
     """Algorithmic work of the two kernels, from the plan: the decode
-    kernel's KV bytes (the blocks its rows read: all of a row's keys, or
-    those after a shared prefix the prefill kernel attends) + q/out of its
-    rows, and the prefill kernel's flops (4 D per (query, visible key) pair
-    and query head, shared-prefix pairs included) and q/out bytes."""
+    kernel's KV bytes (the keys its rows attend: all of a row's keys, or
+    those after a shared prefix the prefill kernel attends; K and V of one
+    kv head per key, no padding of a row's last block) + q/out of its rows,
+    and the prefill kernel's flops (4 D per (query, visible key) pair and
+    query head, shared-prefix pairs included)."""
     Hq, D = lay.num_q_heads, lay.head_dim
     dec = lay.q_lens <= 16
     dec_tokens = int(lay.q_lens[dec].sum())
-    kv_dec = int(info["decode_kv_blocks"]) * 16 * D * 2 * 2
+    kv_dec = int(info["decode_kv_keys"]) * D * 2 * 2
     flops = 4 * D * Hq * int(info["prefill_causal_pairs"])
     return {"decode_bytes": kv_dec + 2 * dec_tokens * Hq * D * 2, "prefill_flops": flops}
 
@@ -355,10 +362,8 @@ def run_ours(args):
 
     def one_step(trace=None, ev=None):
         flush.fill_(1)
-        t0 = time.perf_counter()
         plan = plan_pool[step_no[0] % 2].rebuild(h_cu, h_sl, dims, h_bt)
         step_no[0] += 1
-        plan_s = time.perf_counter() - t0
         if ev is not None:
             ev[0].record(stream)
         if trace is not None or args.two_calls:  # the traced entry point is the two-call one
@@ -370,7 +375,7 @@ def run_ours(args):
                                      plan, ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        return plan, plan_s
+        return plan
 
     for _ in range(args.warmup):
         one_step()
@@ -383,12 +388,10 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    plans, plan_times = [], []
+    plans = []
     wall0 = time.perf_counter()
     for i in range(args.steps):
-        plan, plan_s = one_step(None, evs[i])
-        plans.append(plan)
-        plan_times.append(plan_s)
+        plans.append(one_step(None, evs[i]))
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - wall0
     if dist is not None:
@@ -467,6 +470,49 @@ def run_ours(args):
     step_roofline = {"t_roofline_ms": t_roof * 1e3, "t_measured_ms": ms_per_step,
                      "frac": t_roof * 1e3 / ms_per_step}
 
+    # host cost of a plan build (and its table upload), on an idle plan
+    torch.cuda.synchronize(dev)
+    plan_build_us = []
+    for i in range(max(20, args.steps)):
+        t0 = time.perf_counter()
+        plan_pool[i % 2].rebuild(h_cu, h_sl, dims, h_bt)
+        plan_build_us.append((time.perf_counter() - t0) * 1e6)
+
+    # the scatter kernel alone: back-to-back launches on distinct copies of
+    # the step's K/V, each writing its own slots in blocks no request owns,
+    # after an L2 flush
+    scatter = None
+    T, Hkv, D = lay.num_tokens, lay.num_kv_heads, lay.head_dim
+    free = np.setdiff1d(np.arange(lay.num_blocks), np.append(lay.used_blocks(), lay.poison_block))
+    need = -(-T // 16)
+    nsets = min(8, len(free) // need) if T else 0
+    if nsets:
+        tok = np.arange(T, dtype=np.int64)
+        sc_slots = [torch.from_numpy(free[s * need:(s + 1) * need].astype(np.int64)[tok // 16] * 16 + tok % 16).to(dev)
+                    for s in range(nsets)]
+        sc_k = [batch.k.clone() for _ in range(nsets)]
+        sc_v = [batch.v.clone() for _ in range(nsets)]
+        sc_ms = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(4)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for s_ in range(nsets):
+                pa.reshape_and_cache(sc_k[s_], sc_v[s_], sc_slots[s_], kc, vc, stream=stream)
+            e1.record(stream)
+            if i >= args.warmup:
+                sc_ms.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in sc_ms) / nsets
+        sc_bytes = 2 * (2 * T * Hkv * D * 2) + T * 8   # k, v read; cache rows written; slots read
+        sc_gbs = sc_bytes / (per_launch_ms * 1e-3) / 1e9
+        scatter = {"bound": "hbm", "kernel": "reshape_and_cache_kernel", "achieved": sc_gbs,
+                   "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
+                   "frac": sc_gbs / peaks["hbm_gbs"], "algorithmic_bytes": sc_bytes, "ms": per_launch_ms,
+                   "how": f"{nsets} back-to-back launches on distinct inputs and slots after an L2 flush, "
+                          "events around all of them"}
+        del sc_k, sc_v, sc_slots
+
     # e2e: public API with host buffers; H2D of the step's inputs, D2H of out
     e2e = None
     if not args.no_e2e:
@@ -489,10 +535,12 @@ def run_ours(args):
         # inputs, plus the plan tables each step's build uploads
         h2d = nbytes + info["table_bytes"]
         d2h = out_host.numel() * out_host.element_size()
-        e_ms = []
+        e_ms, e_wall_ms, e_ev_ms = [], [], []
         for i in range(args.warmup + args.steps):
             flush.fill_(2)
+            torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0 = time.perf_counter()
             e0.record(stream)
             d_stage.copy_(h_stage, non_blocking=True)
             plan = plan_pool[i % 2].rebuild(h_cu, h_sl, dims, h_bt)
@@ -507,13 +555,19 @@ def run_ours(args):
             out_host.copy_(out, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
+            wall_ms = (time.perf_counter() - t0) * 1e3
             if i >= args.warmup:
-                e_ms.append(e0.elapsed_time(e1))
+                ev_ms = e0.elapsed_time(e1)
+                e_wall_ms.append(wall_ms)
+                e_ev_ms.append(ev_ms)
+                e_ms.append(max(wall_ms, ev_ms))
         e_total = max_over_ranks(sum(e_ms), dist, dev)
         e_val = (world * acct["total"] * args.steps / (e_total * 1e-3) / 1e9) if decode else \
             (world * lay.num_tokens * args.steps / (e_total * 1e-3))
         e2e = {"value": e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_total / args.steps}
+               "ms_per_step": e_total / args.steps,
+               "host_ms_per_step": statistics.mean(e_wall_ms), "events_ms_per_step": statistics.mean(e_ev_ms),
+               "includes": "plan build and table upload, H2D of inputs, scatter + attention, D2H of out"}
 
     # KV export / import of every request's whole history (the local half of
     # moving a request's KV between instances), each call timed alone with
@@ -570,17 +624,21 @@ def run_ours(args):
                        "kv_bytes_logical_per_step": lay.kv_bytes_logical(),
                        "tokens_per_step": lay.num_tokens,
                        "l2": "flushed before every timed step (1 GiB write, outside the events)",
-                       "plan_us_host": 1e6 * statistics.median(plan_times),
+                       "plan_us_host": statistics.median(plan_build_us),
+                       "plan_us_host_note": "pa_plan_build on an idle plan (host partition + table upload), "
+                                            "median",
                        "step_api": ("pa_reshape_and_cache + pa_attention_varlen" if args.two_calls
                                     else "pa_reshape_and_attention"),
                        "stages_ms": {"plan_wait": wait_ms, "decode": dec_ms, "combine": comb_ms,
                                      "prefill": prefill_ms,
+                                     "scatter": scatter["ms"] if scatter else None,
                                      "note": "separate traced passes; event records add GPU time"},
                        "parallelism": f"replicas x{world} (weak: one batch per GPU)",
                        "wall_s_timed_region": wall},
             "roofline": roofline,
             "roofline_decode": roofline_decode,
             "roofline_prefill": roofline_prefill,
+            "roofline_scatter": scatter,
             "kv_transfer": kv_transfer,
             "step_roofline": step_roofline,
             "cpu_baseline": cpu,

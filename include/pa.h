@@ -177,6 +177,10 @@ typedef struct {
     int32_t num_prefix_groups;    /* shared-prefix runs found (h_block_tables given) */
     int32_t attention_launches;   /* kernels one pa_attention_varlen call launches
                                      (decode, staging, prefill, merge) */
+    int64_t decode_kv_keys;       /* sum over decode rows of the keys the split-KV
+                                     kernel attends (a row's keys, less a shared
+                                     prefix the prefill kernel attends); unlike
+                                     decode_kv_blocks, no padding of last blocks */
 } pa_plan_info;
 int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
 
@@ -379,21 +383,53 @@ int pa_validate_inputs(const int64_t *d_slot_mapping, const int32_t *d_block_tab
  *     array's device address with cudaGetSymbolAddress and caches it; make
  *     that first call before any stream capture.  A failed lookup returns
  *     PA_ERR_CUDA.
+ *   - The address is looked up again when the device's current CUDA context
+ *     is another one than at the lookup (after cudaDeviceReset, say, the
+ *     library's device image is loaded anew); the first call in a new
+ *     context must then also come before any stream capture.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents.  Its first word is a status word like a workspace's (zero
- *     at load; the kernels only ever set error bits in it, and its address
- *     is not exposed, so it is not read or cleared).  The rest is scratch
- *     that every call writes before reading; the plan's tables live with
- *     the plan.  Calls
- *     whose GPU work overlaps in time (two streams, or two threads' streams)
- *     race on the array and give undefined results; order them, or use
- *     pa_attention_varlen with separate workspaces.
+ *     at load; the kernels only ever set error bits in it, which
+ *     accumulate until cleared): read and clear it with pa_noalloc_status.
+ *     The rest is scratch that every call writes before reading; the plan's
+ *     tables live with the plan.  Calls whose GPU work overlaps in time (two
+ *     streams, or two threads' streams) race on the array and give
+ *     undefined results; order them, or use pa_attention_varlen with
+ *     separate workspaces.
  */
 size_t pa_noalloc_scratch_bytes(void);
 int pa_attention_varlen_noalloc(const void *d_q, const void *d_k_cache, const void *d_v_cache,
                                 const int32_t *d_block_tables, const int32_t *d_cu_seqlens_q,
                                 const int32_t *d_seq_lens, float scale, void *d_out,
                                 const pa_dims *dims, const pa_plan *plan, void *stream);
+
+/*
+ * Status word of the no-alloc array on the current device, the counterpart
+ * of pa_workspace_status for pa_attention_varlen_noalloc: copies the word to
+ * *status after the work queued on `stream` before it (the call waits for
+ * `stream`), and with clear != 0 then zeroes it (queued on `stream`, done
+ * before the call returns).  0 means no error; bit 0 means some bounded wait
+ * inside a kernel of a no-alloc call gave up (that call's output is
+ * undefined).  Allocates nothing.  Like the no-alloc call itself, it races
+ * with no-alloc work queued on other streams.
+ * Errors: PA_ERR_NULL, PA_ERR_CUDA.
+ */
+int pa_noalloc_status(uint32_t *status, int clear, void *stream);
+
+/*
+ * Self-test of the bounded-wait error path.  Every mbarrier wait in the
+ * tensor-core kernels gives up after a limit (about a second) and sets bit 0
+ * of the status word; this call makes such a wait run out on purpose, with
+ * nothing else in flight: it queues on `stream` a one-CTA kernel that holds
+ * tensor memory, waits limit_cycles SM cycles on an mbarrier that nothing
+ * arrives at, sets bit 0 of the word at d_workspace (a workspace or any
+ * 256-byte aligned device word) and releases the tensor memory.  Read the
+ * result with pa_workspace_status and clear it with pa_workspace_reset.
+ * The pages have no counterpart: it checks the library's failure reporting.
+ * Errors: PA_ERR_NULL, PA_ERR_WORKSPACE (misaligned), PA_ERR_SHAPE
+ * (limit_cycles outside 1 .. 2e9), PA_ERR_CUDA.
+ */
+int pa_selftest_wait_timeout(void *d_workspace, long long limit_cycles, void *stream);
 
 /* Static text for a status code. */
 const char *pa_status_string(int status);

@@ -26,7 +26,8 @@ __all__ = ["load_library", "library_path", "PaError", "Dims", "dims_of", "Plan",
            "workspace_for",
            "PA_OK", "PA_ERR_NULL", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "PA_ERR_ALIGN",
            "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE", "PA_ERR_BOUNDS", "PA_ERR_CUDA", "PA_ERR_PLAN",
-           "PA_ERR_TOO_LARGE", "attention_varlen_noalloc", "noalloc_scratch_bytes", "workspace_status"]
+           "PA_ERR_TOO_LARGE", "attention_varlen_noalloc", "noalloc_scratch_bytes", "noalloc_status",
+           "workspace_status", "workspace_reset", "selftest_wait_timeout"]
 
 PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE, PA_ERR_ALIGN = 0, -1, -2, -3, -4
 PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_BOUNDS, PA_ERR_CUDA, PA_ERR_PLAN = -5, -6, -7, -8, -9
@@ -66,7 +67,8 @@ class PlanInfo(ctypes.Structure):
                 ("decode_kv_blocks", ctypes.c_int64), ("prefill_causal_pairs", ctypes.c_int64),
                 ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
                 ("num_staged_kv_tiles", ctypes.c_int32), ("num_prefill_ctas", ctypes.c_int32),
-                ("num_prefix_groups", ctypes.c_int32), ("attention_launches", ctypes.c_int32)]
+                ("num_prefix_groups", ctypes.c_int32), ("attention_launches", ctypes.c_int32),
+                ("decode_kv_keys", ctypes.c_int64)]
 
     def as_dict(self):
         return {n: int(getattr(self, n)) for n, _ in self._fields_}
@@ -99,6 +101,8 @@ def load_library():
             "pa_noalloc_scratch_bytes": (SZ, []),
             "pa_workspace_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "pa_workspace_reset": (I, [P, P, P]),
+            "pa_noalloc_status": (I, [ctypes.POINTER(ctypes.c_uint32), I, P]),
+            "pa_selftest_wait_timeout": (I, [P, ctypes.c_longlong, P]),
             "pa_validate_scratch_bytes": (SZ, [DP]),
             "pa_validate_inputs": (I, [P, P, P, P, DP, P, SZ, P]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -379,6 +383,22 @@ def workspace_reset(workspace: torch.Tensor, plan: "Plan", stream=None) -> None:
     """Zero a workspace's status word and merge tickets (after an error)."""
     _check(load_library().pa_workspace_reset(_dev_ptr(workspace, "workspace"), plan.handle, _stream_ptr(stream)),
            "pa_workspace_reset")
+
+
+def noalloc_status(clear: bool = False, stream=None) -> int:
+    """Error bits in the no-alloc array's status word on the current device
+    (0 = none); with clear, zero the word afterwards.  Waits for the stream."""
+    st = ctypes.c_uint32(0)
+    _check(load_library().pa_noalloc_status(ctypes.byref(st), 1 if clear else 0, _stream_ptr(stream)),
+           "pa_noalloc_status")
+    return int(st.value)
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_cycles: int, stream=None) -> None:
+    """Queue the bounded-wait self-test: a kernel whose mbarrier wait runs out
+    after limit_cycles sets bit 0 of the workspace's status word."""
+    _check(load_library().pa_selftest_wait_timeout(_dev_ptr(workspace, "workspace"), int(limit_cycles),
+                                                   _stream_ptr(stream)), "pa_selftest_wait_timeout")
 
 
 def noalloc_scratch_bytes() -> int:

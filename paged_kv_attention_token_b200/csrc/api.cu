@@ -94,7 +94,7 @@ extern "C" int pa_reshape_and_cache(const void *k, const void *v, const int64_t 
         k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
         (int64_t)d.num_blocks * d.block_size, current_sm_count(),
         static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return e == cudaSuccess ? PA_OK : cuda_error();
 }
 
 namespace {
@@ -176,14 +176,14 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const uint8_t *tb = static_cast<const uint8_t *>(plan->d_tables);
-    if (mark(trace, 0, stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (mark(trace, 0, stream) != cudaSuccess) return cuda_error();
     // The plan's tables are on the device since its build returned, so
     // nothing sits between the caller's previous kernel and the decode
     // kernel's programmatic launch.  Under stream capture (a CUDA graph) the
     // plan-use event below is not recorded: a graph replay is not tracked by
     // the plan, whose rebuild then must not overlap one.
     cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) return cuda_error();
     const bool track_use = capture == cudaStreamCaptureStatusNone;
     const float scale_log2 = scale * kLog2e;
     DecodeParams p{};
@@ -239,6 +239,7 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         pp.group = plan->group;
         pp.max_blocks_per_seq = d.max_blocks_per_seq;
         pp.scale_log2 = scale_log2;
+        pp.wait_limit = kWaitLimitCycles;
     }
     const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
     if (side_by_side) {
@@ -248,56 +249,56 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         // sized for the other SMs, waits on a side stream of the least
         // priority for the fork event and fills those SMs.
         cudaStream_t side = side_stream(plan->device);
-        if (!side) return PA_ERR_CUDA;
+        if (!side) return cuda_error();
         cudaEvent_t fork = static_cast<cudaEvent_t>(plan->fork_event);
         cudaEvent_t join = static_cast<cudaEvent_t>(plan->join_event);
-        if (mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (cudaEventRecord(fork, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (cudaStreamWaitEvent(side, fork, 0) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 1, side) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
+        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (cudaEventRecord(fork, stream) != cudaSuccess) return cuda_error();
+        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (cudaStreamWaitEvent(side, fork, 0) != cudaSuccess) return cuda_error();
+        if (mark(trace, 1, side) != cudaSuccess) return cuda_error();
         // shared-prefix partials are not ready while the decode kernel runs:
         // it leaves every merge to the merge kernel after the join
         p.defer_merge = plan->cascade ? 1 : 0;
-        if (launch_decode(p, d.head_dim, side) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 2, side) != cudaSuccess || mark(trace, 3, side) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;  // prefill, not the join
+        if (launch_decode(p, d.head_dim, side) != cudaSuccess) return cuda_error();
+        if (mark(trace, 2, side) != cudaSuccess || mark(trace, 3, side) != cudaSuccess) return cuda_error();
+        if (mark(trace, 5, stream) != cudaSuccess) return cuda_error();  // prefill, not the join
         if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
-            return PA_ERR_CUDA;
+            return cuda_error();
         if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
-            return PA_ERR_CUDA;
+            return cuda_error();
         if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
-            return PA_ERR_CUDA;
+            return cuda_error();
         return PA_OK;
     } else if (plan->cascade) {
         // shared-prefix partials first; the decode kernel merges them
-        if (mark(trace, 4, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 5, stream) != cudaSuccess || mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
+        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (mark(trace, 5, stream) != cudaSuccess || mark(trace, 1, stream) != cudaSuccess) return cuda_error();
+        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess) return cuda_error();
         if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
-            return PA_ERR_CUDA;
+            return cuda_error();
         return PA_OK;
     } else {
-        if (mark(trace, 1, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (mark(trace, 1, stream) != cudaSuccess) return cuda_error();
         // right behind the step's own scatter (fused step, no trace events)
         p.wait_first = k_new != nullptr && !trace ? 0 : 1;
-        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+        if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
         if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess ||
             mark(trace, 4, stream) != cudaSuccess)
-            return PA_ERR_CUDA;
+            return cuda_error();
         if (plan->num_tiles > 0) {
-            if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
-            if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return PA_ERR_CUDA;
+            if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+            if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         }
     }
-    if (mark(trace, 5, stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (mark(trace, 5, stream) != cudaSuccess) return cuda_error();
     // the plan's next build waits for this
     if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
-        return PA_ERR_CUDA;
+        return cuda_error();
     return PA_OK;
 }
 }  // namespace
@@ -332,7 +333,7 @@ extern "C" int pa_reshape_and_attention(const void *k, const void *v, const int6
     if (launch_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
                                  (int64_t)d.num_blocks * d.block_size, current_sm_count(),
                                  static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return PA_ERR_CUDA;
+        return cuda_error();
     return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, d, plan,
                            workspace, stream, nullptr, k, v);
 }
@@ -356,7 +357,7 @@ int kv_transfer(bool do_export, const void *src_k, const void *src_v, void *dst_
                                              d.num_seqs, d.max_blocks_per_seq, d.num_blocks, d.num_tokens,
                                              d.num_kv_heads * d.head_dim, current_sm_count(),
                                              static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return e == cudaSuccess ? PA_OK : cuda_error();
 }
 }  // namespace
 
@@ -376,7 +377,7 @@ extern "C" int pa_workspace_reset(void *workspace, const pa_plan *plan, void *st
     if (!workspace || !plan) return PA_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign) return PA_ERR_WORKSPACE;
     if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream_)) != cudaSuccess)
-        return PA_ERR_CUDA;
+        return cuda_error();
     return PA_OK;
 }
 
@@ -385,7 +386,7 @@ extern "C" int pa_workspace_status(const void *workspace, void *stream_, uint32_
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
-        return PA_ERR_CUDA;
+        return cuda_error();
     return PA_OK;
 }
 
@@ -482,10 +483,10 @@ extern "C" int pa_validate_inputs(const int64_t *slot_mapping, const int32_t *bl
     const size_t words = ((size_t)d.num_blocks * d.block_size + 31) / 32;
     if (launch_validate(slot_mapping, block_tables, cu_seqlens_q, seq_lens, d, bitmap, words, flag,
                         stream) != cudaSuccess)
-        return PA_ERR_CUDA;
+        return cuda_error();
     uint32_t h_flag = 0;
     if (cudaMemcpyAsync(&h_flag, flag, sizeof h_flag, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-        return PA_ERR_CUDA;
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+        return cuda_error();
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return cuda_error();
     return h_flag ? PA_ERR_BOUNDS : PA_OK;
 }

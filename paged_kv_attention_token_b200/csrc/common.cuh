@@ -89,9 +89,9 @@ __device__ __forceinline__ float warp_max_xor(float v, int lane_mask) {
 // ---------------------------------------------------------------------------
 namespace pa {
 
-// A wait on an mbarrier gives up after this many SM cycles (about a second at
-// B200 clocks); the kernel then records an error and finishes without
-// waiting further.
+// A wait on an mbarrier gives up after this many SM cycles by default (about
+// a second at B200 clocks); the kernel then records an error and finishes
+// without waiting further.  Kernels take the limit as a parameter.
 constexpr long long kWaitLimitCycles = 2000000000ll;
 
 // Error bits a kernel can set in the workspace status word.
@@ -132,12 +132,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase of `parity` to complete; false if it did not within
-// kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// `limit` SM cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     return true;
 }
 

@@ -73,11 +73,17 @@ struct PrefillParams {
     int group;
     int max_blocks_per_seq;
     float scale_log2;
+    long long wait_limit;  // SM cycles an mbarrier wait may take before the kernel gives up
 };
 
 // Gathers the staged K/V tiles (must precede launch_prefill in stream order).
 cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream);
+
+// Self-test of the bounded-wait error path: one CTA holds tensor memory,
+// waits on an mbarrier that nothing arrives at for `limit` cycles, records
+// kStatusWaitTimeout in *status and releases the tensor memory.
+cudaError_t launch_wait_selftest(uint32_t *status, long long limit, cudaStream_t stream);
 
 // Data-dependent precondition checks; writes a nonzero flag word on failure.
 cudaError_t launch_validate(const int64_t *slots, const int32_t *block_tables,

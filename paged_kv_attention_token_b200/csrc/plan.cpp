@@ -279,12 +279,12 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     const bool fresh = (p == nullptr);
     if (fresh) {
         p = new (std::nothrow) pa_plan();
-        if (!p) return PA_ERR_CUDA;
+        if (!p) return pa::cuda_error();
         p->device = device;
         if (!create_sync_objects(p)) {
             cudaGetLastError();
             pa_plan_destroy(p);
-            return PA_ERR_CUDA;
+            return pa::cuda_error();
         }
     } else if (p->device != device) {
         return PA_ERR_PLAN;
@@ -489,6 +489,8 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     p->num_pieces = piece_base;
     p->num_combine = (int32_t)combine.size();
     p->decode_blocks = total;
+    p->decode_keys = 0;
+    for (const pa::DecodeRow &r : rows) p->decode_keys += r.n_keys - (int64_t)r.first_block * pa::kBlockSize;
     p->num_tiles = (int32_t)tiles.size();
     p->num_prefill_ctas = grid;
     p->num_stages = (int32_t)stages.size();
@@ -522,7 +524,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     }
     if (!reserve_tables(p, t.bytes)) {
         if (fresh) pa_plan_destroy(p);
-        return PA_ERR_CUDA;
+        return pa::cuda_error();
     }
     std::memset(p->tables, 0, t.bytes);
     std::memcpy(p->tables + t.units, units.data(), sizeof(pa::DecodeUnit) * units.size());
@@ -538,7 +540,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     if (!upload_tables(p)) {
         cudaGetLastError();
         if (fresh) pa_plan_destroy(p);
-        return PA_ERR_CUDA;
+        return pa::cuda_error();
     }
     *out = p;
     return PA_OK;
@@ -562,6 +564,7 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     // as pa_attention_varlen launches them: the decode kernel; staging and
     // prefill; the merge kernel when shared-prefix tiles run beside decode
     const bool side_by_side = p->overlap_sms > 0 && p->num_units > 0 && p->num_tiles > 0;
+    info->decode_kv_keys = p->decode_keys;
     info->attention_launches = (p->num_units > 0 ? 1 : 0) + (p->num_tiles > 0 ? 1 : 0) +
                                (p->num_tiles > 0 && p->num_stages > 0 ? 1 : 0) +
                                (side_by_side && p->cascade && p->num_combine > 0 ? 1 : 0);

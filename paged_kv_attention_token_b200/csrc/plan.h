@@ -7,9 +7,19 @@
 #include <cstdint>
 #include <vector>
 
+#include <cuda_runtime.h>
+
 #include "../../include/pa.h"
 
 namespace pa {
+
+// PA_ERR_CUDA, after clearing the calling thread's last CUDA error, so that
+// the failure is reported once and a later call's launch check does not
+// see it again.
+inline int cuda_error() {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+}
 
 constexpr int kBlockSize = 16;
 // Segments with q_len above this go to the tensor-core prefill kernel; the
@@ -130,7 +140,8 @@ struct pa_plan {
     int32_t num_rows = 0;
     int32_t num_pieces = 0;
     int32_t num_combine = 0;
-    int64_t decode_blocks = 0;           // sum over rows of ceil(n_keys / 16)
+    int64_t decode_blocks = 0;           // sum over rows of ceil(n_keys / 16) - first_block
+    int64_t decode_keys = 0;             // sum over rows of n_keys - 16 first_block
     // prefill part
     int32_t num_tiles = 0;
     int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)

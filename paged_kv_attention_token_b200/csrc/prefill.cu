@@ -215,7 +215,7 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
     float m = -INFINITY, l = 0.f;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
     for (int j = 0; j < nkv; ++j, ++it) {
-        if (!err && !mbar_wait(s_full, it & 1)) err = true;
+        if (!err && !mbar_wait(s_full, it & 1, p.wait_limit)) err = true;
         tc_fence_after();
         const int kbase = 128 * (kv_tile0 + j);  // first key of this step
         // only tiles that reach past the first query's position need the
@@ -276,7 +276,7 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         f2_split(lsum, l0, l1);
         l = l * alpha + (l0 + l1);
     }
-    if (!err && !mbar_wait(o_done, k & 1)) err = true;
+    if (!err && !mbar_wait(o_done, k & 1, p.wait_limit)) err = true;
     tc_fence_after();
     // the whole O row at once (one wait: TMEM loads queue behind the MMAs of
     // the other head), then O is free for the next tile
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(384, 1)
                                  kk > 0 ? 1u : acc0);
             };
             auto wait = [&](uint64_t *bar, uint32_t parity) {
-                if (!err && !mbar_wait(bar, parity)) err = true;
+                if (!err && !mbar_wait(bar, parity, p.wait_limit)) err = true;
             };
             int vs = 0, ks = 0;          // ring slots of the next V and K tiles
             uint32_t vph = 0, kph = 0;   // and their phases
@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int nkv = tile.n_kv_tiles;
                 const int hA = tile.head;
                 const int tok0 = tile.row_base >= 0 ? tile.q_start : p.cu_seqlens_q[tile.seq] + tile.q_start;
-                if (ti > t_begin && !err && !mbar_wait(q_empty, (uint32_t)(ti - t_begin - 1) & 1)) err = true;
+                if (ti > t_begin && !err && !mbar_wait(q_empty, (uint32_t)(ti - t_begin - 1) & 1, p.wait_limit)) err = true;
                 mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < C::kSlabs; ++s) {
@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint8_t *kv_tiles = p.staged + (size_t)(tile.kv_base + tile.kv_tile0) * 2 * C::kTileBytes;
                 auto load_k = [&](int j) {
                     if (kuse >= (uint32_t)C::kKStages && !err &&
-                        !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1))
+                        !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1, p.wait_limit))
                         err = true;
                     mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
                     bulk_load(sK + ks * C::kTileBytes, kv_tiles + (size_t)j * 2 * C::kTileBytes, C::kTileBytes,
@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(384, 1)
                 };
                 auto load_v = [&](int j) {
                     if (vuse >= (uint32_t)C::kVStages && !err &&
-                        !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1))
+                        !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1, p.wait_limit))
                         err = true;
                     mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
                     bulk_load(sV + vs * C::kTileBytes, kv_tiles + ((size_t)j * 2 + 1) * C::kTileBytes, C::kTileBytes,

@@ -44,6 +44,8 @@ int main(void) {
     CHECK(3, info.num_decode_rows == 16);
     /* blocks the rows read: ceil(17/16) + ceil(40/16) + sum_j ceil((j+1)/16) for j < 6, per kv head */
     CHECK(4, info.decode_kv_blocks == (2 + 3 + 6) * 2);
+    /* keys without last-block padding: 17 + 40 + (1 + 2 + ... + 6), per kv head */
+    CHECK(4, info.decode_kv_keys == (17 + 40 + 21) * 2);
     CHECK(5, info.num_prefill_tiles == 0 && info.num_sms == 148);
     CHECK(6, pa_plan_workspace_bytes(plan) == info.workspace_bytes && info.workspace_bytes >= 256);
     CHECK(7, info.attention_launches == 1);

@@ -22,3 +22,16 @@ def cuda_lib():
     import paged_kv_attention_token_b200 as pa
     pa.load_library()
     return pa
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Errors of every parity comparison the session made (GPU tests)."""
+    from tests import parity
+    if not parity.RECORDS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", f"parity against the oracle ({len(parity.RECORDS)} comparisons; "
+                      f"bar: max |err| <= {parity.MAX_ABS}, mean |err| <= {parity.MEAN_ABS})")
+    for what, n, e in parity.RECORDS:
+        tr.write_line(f"{what[:60]:<60} values {n:>9}  max {e['max_abs']:.2e}  mean {e['mean_abs']:.2e}  "
+                      f"max_rel {e['max_rel']:.2e}  nan {e['nan']}")

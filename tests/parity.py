@@ -1,9 +1,15 @@
 """Parity bar shared by the tests: bf16 attention output, converted to fp32,
-against the fp64 oracle: max |err| <= 2e-2 and mean |err| <= 2e-3."""
+against the fp64 oracle: max |err| <= 2e-2 and mean |err| <= 2e-3.
+
+Every comparison is recorded (case name, rows compared, max / mean absolute
+and max relative error); tests/conftest.py prints the records at the end of
+the session, so a quiet run still shows how far each case is from the bar."""
 import numpy as np
 
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
+
+RECORDS = []
 
 
 def errors(got, want):
@@ -24,5 +30,6 @@ def within(got, want) -> bool:
 
 def assert_parity(got, want, what=""):
     e = errors(got, want)
+    RECORDS.append((what, int(np.asarray(want).size), e))
     assert e["nan"] == 0 and e["max_abs"] <= MAX_ABS and e["mean_abs"] <= MEAN_ABS, f"{what}: {e}"
     return e

@@ -65,11 +65,13 @@ def test_plan_invariants(lib, name):
     # one row per (decode query, kv head); its keys are its causal prefix
     rows = int(ql[dec].sum()) * lay.num_kv_heads
     assert info["num_decode_rows"] == rows
-    blocks = 0
+    blocks = keys = 0
     for L, n in zip(ql[dec], sl[dec]):
         for j in range(L):
             blocks += -(-(n - L + j + 1) // 16)
+            keys += n - L + j + 1
     assert info["decode_kv_blocks"] == blocks * lay.num_kv_heads
+    assert info["decode_kv_keys"] == keys * lay.num_kv_heads
     # one wave of warps at most (12 per SM at D=64, 8 at D=128), each with a
     # fair share of at least 4 blocks
     warps_per_sm = 12 if lay.head_dim == 64 else 8
@@ -221,6 +223,13 @@ def test_compute_calls_reject_bad_arguments_before_any_launch(lib):
         assert fn(fake, fake, fake, fake, fake, fake, ctypes.byref(dk), S) == pa.PA_ERR_SHAPE  # rows, no requests
     # validate: scratch too small
     assert lib.pa_validate_inputs(fake, fake, fake, fake, ctypes.byref(d), fake, 8, S) == pa.PA_ERR_WORKSPACE
+    # bounded-wait self-test: status word missing or misaligned, limit out of range
+    assert lib.pa_selftest_wait_timeout(None, 1000, S) == pa.PA_ERR_NULL
+    assert lib.pa_selftest_wait_timeout(ctypes.c_void_p(0x10010), 1000, S) == pa.PA_ERR_WORKSPACE
+    assert lib.pa_selftest_wait_timeout(fake, 0, S) == pa.PA_ERR_SHAPE
+    assert lib.pa_selftest_wait_timeout(fake, 3 * 10 ** 9, S) == pa.PA_ERR_SHAPE
+    # no-alloc status word: nowhere to put it
+    assert lib.pa_noalloc_status(None, 0, S) == pa.PA_ERR_NULL
 
 
 def test_status_strings(lib):
@@ -325,6 +334,8 @@ def test_shared_prefix_detection_on_constructed_tables(lib):
     dec = [(n, sh) for L, n, _, sh in segs if L == 1]
     assert without["decode_kv_blocks"] == sum(-(-n // 16) for n, _ in dec) * Hkv
     assert with_tables["decode_kv_blocks"] == sum(-(-n // 16) - sh for n, sh in dec) * Hkv
+    assert without["decode_kv_keys"] == sum(n for n, _ in dec) * Hkv
+    assert with_tables["decode_kv_keys"] == sum(n - 16 * sh for n, sh in dec) * Hkv
     # the prefix tiles join the prefill segment's tiles and pairs
     assert with_tables["num_prefill_tiles"] > without["num_prefill_tiles"]
     extra_pairs = (6 * 20 + 5 * 16) * 16

@@ -63,6 +63,12 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_lib):
             torch.cuda.synchronize()
             assert_parity(out.float().cpu().numpy(), ref.float().cpu().numpy().astype(np.float64),
                           f"no-alloc call {rnd} ({b.layout.name})")
+    # the array's status word: no bounded wait ran out in any of the calls;
+    # reading it with clear leaves it zero
+    st = ctypes.c_uint32(7)
+    assert lib.pa_noalloc_status(ctypes.byref(st), 1, None) == pa.PA_OK
+    assert st.value == 0
+    assert pa.noalloc_status() == 0
 
 
 def test_noalloc_rejects_plans_beyond_its_array(cuda_lib):
