@@ -65,6 +65,18 @@ namespace {
 
 constexpr float kPrefillRescaleThreshold = 8.f;
 
+// The softmax evaluates 2^x on two pipes: the MUFU unit (ex2.approx) and, for
+// the pairs k (0..15) of a 32-column chunk with bit k % 4 set in
+// kPolyPairMask, a polynomial on the FMA and integer pipes.  The MUFU unit
+// does 16 results per SM clock, so 128 x 128 exponentials per head and
+// 128-key step take as long as that step's MMAs; moving part of them to the
+// FMA pipe shortens each softmax chain.
+constexpr uint32_t kPolyPairMask = 0x0;
+// P is packed to bf16 pairs either with cvt.rn.bf16x2.f32 or with integer
+// adds and a byte permute (rounding half up; it differs from round-to-even
+// only on exact ties).
+constexpr bool kPackOnAlu = false;
+
 template <int D>
 struct PrefillCfg {
     static constexpr int kThreads = 384;
@@ -134,6 +146,54 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x of a pair without the MUFU unit.  With x clamped to >= -127,
+// 2^x = 2^n * 2^f for n = floor(x) and f = x - n in [0, 1): adding 1.5 * 2^23
+// with rounding toward -inf leaves n in the low mantissa bits of the sum (so
+// n is exact and f = x - n exact), 2^f is a cubic in f, and 2^n enters by
+// adding n to the exponent field of the cubic's value (the low bits of the
+// sum, shifted up 23 places, are n mod 2^9).  The cubic's coefficients were
+// fitted here to 2^f on [0, 1) by least squares reweighted towards the
+// smallest maximum relative error: 8.6e-5, against 2^-9 for the bf16 P the
+// value becomes.  At x = -127 the result is about 2^-127 (masked keys are
+// zeroed by selection).
+__device__ __forceinline__ uint64_t exp2_poly(uint64_t x) {
+    constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+    constexpr float kC1 = 0.6951165795326233f, kC2 = 0.22764593362808228f, kC3 = 0.07706617563962936f;
+    float x0, x1;
+    f2_split(x, x0, x1);
+    x = f2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t magic = f2(kMagic, kMagic);
+    const uint64_t t = f2_add_rm(x, magic);
+    const uint64_t fr = f2_sub(x, f2_sub(t, magic));
+    uint64_t p = f2_fma(fr, f2(kC3, kC3), f2(kC2, kC2));
+    p = f2_fma(fr, p, f2(kC1, kC1));
+    p = f2_fma(fr, p, f2(1.f, 1.f));
+    float p0, p1, t0, t1;
+    f2_split(p, p0, p1);
+    f2_split(t, t0, t1);
+    return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+              __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// bf16 pair of two probabilities (>= 0): e0 in the low half.
+__device__ __forceinline__ uint32_t pack_p(float e0, float e1) {
+    if constexpr (kPackOnAlu) {
+        return __byte_perm(__float_as_uint(e0) + 0x8000u, __float_as_uint(e1) + 0x8000u, 0x7632);
+    } else {
+        return pack_bf16x2(e0, e1);
+    }
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -160,23 +220,31 @@ __device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], bool masked,
     return fmaxf(a, b);
 }
 
-// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs.
-// (Evaluating part of the exponentials on the FMA pipe with a polynomial,
-// or all of them as f16 pairs, was measured slower here: the softmax is
-// bound by the latency and count of its instructions, not by the MUFU unit.)
+// P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; keys past
+// `pos` (when `masked`) get P = 0 by selection.
 __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t scale2,
                                           uint64_t nm2, bool masked, int key0, int pos) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
-        float x0, x1;
-        f2_split(x, x0, x1);
-        if (masked) {
-            if (key0 + 2 * c > pos) x0 = -INFINITY;
-            if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
+        float e0, e1;
+        if ((kPolyPairMask >> (c & 3)) & 1u) {
+            f2_split(exp2_poly(x), e0, e1);
+            if (masked) {
+                if (key0 + 2 * c > pos) e0 = 0.f;
+                if (key0 + 2 * c + 1 > pos) e1 = 0.f;
+            }
+        } else {
+            float x0, x1;
+            f2_split(x, x0, x1);
+            if (masked) {
+                if (key0 + 2 * c > pos) x0 = -INFINITY;
+                if (key0 + 2 * c + 1 > pos) x1 = -INFINITY;
+            }
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
         }
-        const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-        pk[c] = pack_bf16x2(e0, e1);
+        pk[c] = pack_p(e0, e1);
     }
 }
 
@@ -265,7 +333,8 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(p_full);
         // the row sum, off the path that hands P to the tensor cores
         regs_after(pk0);
         regs_after(pk1);
@@ -285,7 +354,8 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
     for (int i = 0; i < D / 32; ++i) tmem_ld32(trow + o_col + 32 * i, o[i]);
     tmem_ld_wait();
     tc_fence_before();
-    mbar_arrive(o_free);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(o_free);
     if (row_base >= 0) {
         // shared-prefix tile: unnormalised O and (max, sum) become one
         // partial of the decode row of this token and kv head (hl: the
@@ -396,12 +466,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(sA_full, 1);
         mbar_init(sB_full, 1);
-        mbar_init(pA_full, 128);
-        mbar_init(pB_full, 128);
+        mbar_init(pA_full, 4);  // one arrive per softmax warp
+        mbar_init(pB_full, 4);
         mbar_init(oA_done, 1);
         mbar_init(oB_done, 1);
-        mbar_init(oA_free, 128);
-        mbar_init(oB_free, 128);
+        mbar_init(oA_free, 4);
+        mbar_init(oB_free, 4);
         fence_mbar_init();
     }
     if (warp == 0) {

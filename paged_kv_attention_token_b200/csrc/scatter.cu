@@ -22,10 +22,12 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
         const int64_t t = c / chunks_per_token;
         const int64_t part = c - t * chunks_per_token;
+        // the chunk's K/V do not depend on the slot: all three loads are in
+        // flight together, and only the stores wait for the slot
         const int64_t s = __ldg(slots + t);
-        if (s < 0 || s >= num_slots) continue;  // negative: skip; past the pool: never written
         const uint4 kv = ld_stream16(k + c);
         const uint4 vv = ld_stream16(v + c);
+        if (s < 0 || s >= num_slots) continue;  // negative: skip; past the pool: never written
         const int64_t dst = s * chunks_per_token + part;
         k_cache[dst] = kv;
         v_cache[dst] = vv;
