@@ -14,11 +14,14 @@ chunked-prefill step with the Qwen2.5-1.5B attention shape (1152 decodes, a
 2048-token chunk on 6144 cached tokens, fresh prompts of 1024/1536/2432).
 
 Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier and
-torch.cuda.synchronize() on both sides.  L2 is flushed (a 1 GiB write)
-before every step and each step's device time is taken with CUDA events on
-the launching stream, excluding the flush; the host plan for a step is built
-and its kernels queued while the flush runs, so the events see device time
-rather than host launch overhead.  Multi-GPU (torchrun): every rank runs its own batch of
+torch.cuda.synchronize() on both sides.  L2 is flushed before every step: a
+1 GiB write, then a read of another 1 GiB buffer, so that a step starts with
+none of its data in L2 and no dirty lines of the flush buffer either (their
+write-back would otherwise be charged to the step's first kernel).  Each
+step's device time is taken with CUDA events on the launching stream,
+excluding the flush; the host plan for a step is built and its kernels
+queued while the flush runs, so the events see device time rather than host
+launch overhead.  Multi-GPU (torchrun): every rank runs its own batch of
 the same shape (weak scaling, no collective on the data path); the reported
 time is the max over ranks.
 
@@ -352,6 +355,13 @@ def run_ours(args):
     info = plan0.info()
     ws = pa.workspace_for(plan0, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def flush_l2(v):
+        """Evict L2: write one buffer larger than L2, then read another (clean lines)."""
+        flush.fill_(v)
+        torch.sum(flush_read, dim=0, out=flush_sink)
     stream = torch.cuda.current_stream(dev)
     # the scatter, then the kernels the attention call launches (plan info)
     launches_per_step = (1 if lay.num_tokens else 0) + info["attention_launches"]  # scatter + attention
@@ -361,7 +371,7 @@ def run_ours(args):
     step_no = [0]
 
     def one_step(trace=None, ev=None):
-        flush.fill_(1)
+        flush_l2(1)
         plan = plan_pool[step_no[0] % 2].rebuild(h_cu, h_sl, dims, h_bt)
         step_no[0] += 1
         if ev is not None:
@@ -494,7 +504,7 @@ def run_ours(args):
         sc_v = [batch.v.clone() for _ in range(nsets)]
         sc_ms = []
         for i in range(args.warmup + args.steps):
-            flush.fill_(4)
+            flush_l2(4)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for s_ in range(nsets):
@@ -537,7 +547,7 @@ def run_ours(args):
         d2h = out_host.numel() * out_host.element_size()
         e_ms, e_wall_ms, e_ev_ms = [], [], []
         for i in range(args.warmup + args.steps):
-            flush.fill_(2)
+            flush_l2(2)
             torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             t0 = time.perf_counter()
@@ -584,7 +594,7 @@ def run_ours(args):
         def time_calls(fn):
             ms = []
             for i in range(args.warmup + args.steps):
-                flush.fill_(3)
+                flush_l2(3)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 fn()
@@ -623,7 +633,7 @@ def run_ours(args):
                        "bytes_per_step": acct["total"], "kv_bytes_per_step": acct["kv"],
                        "kv_bytes_logical_per_step": lay.kv_bytes_logical(),
                        "tokens_per_step": lay.num_tokens,
-                       "l2": "flushed before every timed step (1 GiB write, outside the events)",
+                       "l2": "flushed before every timed step (1 GiB write, then 1 GiB read; outside the events)",
                        "plan_us_host": statistics.median(plan_build_us),
                        "plan_us_host_note": "pa_plan_build on an idle plan (host partition + table upload), "
                                             "median",

@@ -136,6 +136,61 @@ int overlap_split(int num_sms, int64_t prefill_steps, int64_t decode_bytes) {
     return best_p;
 }
 
+// Key splits of the shared prefixes and SMs of the prefill kernel beside the
+// decode kernel, chosen together for plans with shared-prefix groups.  Each
+// group's prefix tiles (chunks x kv heads x head pairs x splits) cost their
+// 128-key tiles plus kPrefixTileOverheadSteps each and are nearly uniform, so
+// dealt to s persistent CTAs they take ceil(tiles / s) tiles' time; other
+// prefill tiles add their average load and one largest tile.  The decode side
+// is costed in the blocks its runs stream plus kRowCostBlocks per row (the
+// charge the run partition uses).  Picks the fastest (splits, SMs), the
+// fewest splits among equals; B200, shared-prefix workload: 2 splits on 64
+// SMs beat 4 on 78 (the old choice; 128 tiles left half the CTAs with two),
+// 2 on 52 or 58, 3, and 1.
+struct CascadeChoice {
+    int splits = 1;
+    int sms = 0;  // 0: the two kernels run one after the other
+};
+
+CascadeChoice choose_cascade(int num_sms, int G, int Hkv, const std::vector<PrefixGroup> &groups,
+                             int64_t other_total, int64_t other_max, int64_t decode_cost_bytes) {
+    CascadeChoice best;
+    double best_us = 1e30;
+    int nt_min = INT32_MAX;
+    for (const PrefixGroup &g : groups) nt_min = std::min<int>(nt_min, (int)cdiv(g.blocks * pa::kBlockSize, pa::kPrefillTileN));
+    auto decode_us = [&](int sms) {
+        return sms <= 0 ? 1e30 : (double)decode_cost_bytes / std::min(kHbmBytesPerUs, sms * kDecodeBytesPerUsPerSm);
+    };
+    for (int sp : {1, 2, 3, 4, 6, 8}) {
+        if (sp > nt_min) break;
+        int64_t tiles = 0, cost = 0;  // prefix tiles and the largest one's cost
+        for (const PrefixGroup &g : groups) {
+            const int64_t nt = cdiv(g.blocks * pa::kBlockSize, pa::kPrefillTileN);
+            tiles += cdiv(g.nseg, pa::kPrefillTileM) * Hkv * cdiv(G, 2) * sp;
+            cost = std::max<int64_t>(cost, cdiv(nt, sp) + kPrefixTileOverheadSteps);
+        }
+        auto prefill_us = [&](int s) {
+            double units = (double)cdiv(tiles, s) * cost;
+            if (other_total > 0) units += (double)other_total / s + (double)other_max;
+            return units * kPrefillStepUs;
+        };
+        // one after the other, on every SM
+        double t = prefill_us(num_sms) + decode_us(num_sms);
+        if (t < best_us) {
+            best_us = t;
+            best = {sp, 0};
+        }
+        for (int s = kMinSideSms; s <= num_sms - kMinSideSms; ++s) {
+            t = std::max(prefill_us(s), decode_us(num_sms - s));
+            if (t < best_us) {
+                best_us = t;
+                best = {sp, s};
+            }
+        }
+    }
+    return best;
+}
+
 // Scoped switch to the plan's device (plans own device memory, a stream and
 // events, which belong to the device they were made on).
 struct DeviceScope {
@@ -345,18 +400,28 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         }
     }
     // Shared-prefix tiles: per group, chunk of up to 128 tokens, kv head,
-    // query-head pair and key split.  The key splits make about one tile per
-    // SM without cutting a split below four 128-key tiles: more splits also
-    // mean more partials for every row to merge (B200: 4 splits of a
-    // 4096-key prefix over 32 base tiles beat 2 and 8).
+    // query-head pair and key split, with the splits (and the SMs the
+    // prefill kernel gets beside the decode kernel) chosen by
+    // choose_cascade.
+    CascadeChoice cascade_choice;
+    if (!groups.empty()) {
+        int64_t other_total = 0, other_max = 0;
+        for (const pa::PrefillTile &t : tiles) {
+            other_total += tile_cost(t);
+            other_max = std::max(other_max, tile_cost(t));
+        }
+        int64_t decode_cost_blocks = 0;
+        for (const pa::DecodeRow &r : rows)
+            decode_cost_blocks += cdiv(r.n_keys, pa::kBlockSize) - r.first_block + kRowCostBlocks;
+        cascade_choice = choose_cascade(p->num_sms, G, Hkv, groups, other_total, other_max,
+                                        decode_cost_blocks * pa::kBlockSize * d.head_dim * 2 * 2);
+    }
     for (size_t k = 0; k < groups.size(); ++k) {
         const PrefixGroup &gr = groups[k];
         const int keys = gr.blocks * pa::kBlockSize;
         const int nt = (int)cdiv(keys, pa::kPrefillTileN);
         const int chunks = (int)cdiv(gr.nseg, pa::kPrefillTileM);
-        const int base_tiles = chunks * Hkv * (int)cdiv(G, 2);
-        const int splits = (int)std::max<int64_t>(
-            1, std::min<int64_t>(cdiv(nt, 4), (int64_t)p->num_sms / base_tiles));
+        const int splits = std::min(cascade_choice.splits, nt);
         group_splits[k] = splits;
         const int base = (int)stages.size();
         for (int g = 0; g < Hkv; ++g)
@@ -388,7 +453,9 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     // merging to a merge kernel after both.
     p->cascade = !groups.empty();
     p->num_prefix_groups = (int32_t)groups.size();
-    p->overlap_sms = overlap_split(p->num_sms, prefill_steps, decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2);
+    p->overlap_sms = groups.empty()
+                         ? overlap_split(p->num_sms, prefill_steps, decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2)
+                         : cascade_choice.sms;
     const int prefill_sms = p->overlap_sms > 0 ? p->overlap_sms : p->num_sms;
     const int decode_sms = p->num_sms - p->overlap_sms;
     const int grid = (int)std::min<size_t>(tiles.size(), (size_t)prefill_sms);

@@ -50,8 +50,9 @@
 //               At the end it reads its O row, divides by its sum and
 //               writes bf16.
 // Every wait is on an mbarrier and bounded; on a timeout the kernel sets a
-// bit in the workspace status word and runs to the end without waiting,
-// after which TMEM is released.
+// bit in the workspace status word and runs to the end without waiting for
+// its partners, but still waits (bounded) for its own MMAs and copies in
+// flight before TMEM is released and the CTA ends.
 #include <cuda.h>
 
 #include <atomic>
@@ -100,7 +101,8 @@ struct PrefillCfg {
     static constexpr int kBarPA = kBarSB + 1, kBarPB = kBarPA + 1;
     static constexpr int kBarOA = kBarPB + 1, kBarOB = kBarOA + 1;
     static constexpr int kBarOAFree = kBarOB + 1, kBarOBFree = kBarOAFree + 1;
-    static constexpr int kNumBars = kBarOBFree + 1;
+    static constexpr int kBarDrain = kBarOBFree + 1;  // every MMA issued has completed
+    static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
     static constexpr int kUsed = kTmemSlotOff + 16;
     // + 1024 to align the base; well above half an SM's shared memory, so
@@ -446,6 +448,7 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *pA_full = bars + C::kBarPA, *pB_full = bars + C::kBarPB;
     uint64_t *oA_done = bars + C::kBarOA, *oB_done = bars + C::kBarOB;
     uint64_t *oA_free = bars + C::kBarOAFree, *oB_free = bars + C::kBarOBFree;
+    uint64_t *drain = bars + C::kBarDrain;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kTmemSlotOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -472,6 +475,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(oB_done, 1);
         mbar_init(oA_free, 4);
         mbar_init(oB_free, 4);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -576,10 +580,12 @@ __global__ void __launch_bounds__(384, 1)
                 ++kA;
                 if (two) ++kB;
             }
-            // nothing of ours may be in flight when TMEM is released: the
-            // last commit on v_empty covers every MMA issued
-            const int last_v = vs == 0 ? C::kVStages - 1 : vs - 1;
-            wait(&v_empty[last_v], vs == 0 ? vph ^ 1u : vph);
+            // nothing of ours may be in flight when TMEM is released: one
+            // more commit covers every MMA issued, and it is waited for even
+            // after a timeout (bounded), so that an error never frees TMEM
+            // under a running MMA
+            umma_commit(drain);
+            if (!mbar_wait(drain, 0, p.wait_limit)) err = true;
         } else if (warp == 1 && lane == 0) {
             // ------------------------------------------------ loads
             int vs = 0, ks = 0;
@@ -625,6 +631,17 @@ __global__ void __launch_bounds__(384, 1)
                     load_v(j);
                 }
             }
+            // every copy has landed before the CTA ends, even after a
+            // timeout (bounded waits): the last load of each stage, the last Q
+            for (int s = 0; s < C::kKStages; ++s) {
+                const uint32_t uses = kuse / C::kKStages + ((uint32_t)s < kuse % C::kKStages ? 1u : 0u);
+                if (uses && !mbar_wait(&k_full[s], (uses - 1) & 1u, p.wait_limit)) err = true;
+            }
+            for (int s = 0; s < C::kVStages; ++s) {
+                const uint32_t uses = vuse / C::kVStages + ((uint32_t)s < vuse % C::kVStages ? 1u : 0u);
+                if (uses && !mbar_wait(&v_full[s], (uses - 1) & 1u, p.wait_limit)) err = true;
+            }
+            if (!mbar_wait(q_full, (uint32_t)(t_end - t_begin - 1) & 1u, p.wait_limit)) err = true;
         }
     } else {
         // ------------------------------------------------ softmax warps
