@@ -516,9 +516,12 @@ def run_ours(args):
         per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in sc_ms) / nsets
         sc_bytes = 2 * (2 * T * Hkv * D * 2) + T * 8   # k, v read; cache rows written; slots read
         sc_gbs = sc_bytes / (per_launch_ms * 1e-3) / 1e9
+        sc_hash = kernel_source_hash(["scatter.cu", "common.cuh", "kernels.h", "plan.h"])
         scatter = {"bound": "hbm", "kernel": "reshape_and_cache_kernel", "achieved": sc_gbs,
                    "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
-                   "frac": sc_gbs / peaks["hbm_gbs"], "algorithmic_bytes": sc_bytes, "ms": per_launch_ms,
+                   "frac": sc_gbs / peaks["hbm_gbs"],
+                   "traffic": profiled_traffic("reshape_and_cache_kernel", args.workload, sc_hash),
+                   "algorithmic_bytes": sc_bytes, "ms": per_launch_ms, "source_hash": sc_hash,
                    "how": f"{nsets} back-to-back launches on distinct inputs and slots after an L2 flush, "
                           "events around all of them"}
         del sc_k, sc_v, sc_slots
