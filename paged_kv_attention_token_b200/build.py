@@ -50,17 +50,19 @@ def _stale(obj: str, src: str, newest_header: float) -> bool:
 # whose sum exceeds what the CTA was launched with would wait forever, so the
 # register count ptxas gives the kernel is checked against the split the
 # source assumes before the library is linked.
-REG_SPLIT_SOURCES = {"prefill.cu": "prefill_kernel"}
+REG_SPLIT_SOURCES = {"prefill.cu": ("prefill_kernel", "prefill_pair_kernel")}
 
 
 def check_register_split(src: str, ptxas_log: str) -> None:
     text = open(src).read()
     want = {k: int(re.search(rf"{k} = (\d+);", text).group(1)) for k in ("kLaunchRegs", "kRegsLow", "kRegsHigh")}
     threads = int(re.search(r"kThreads = (\d+);", text).group(1))
-    kernel = REG_SPLIT_SOURCES[os.path.basename(src)]
-    found = re.findall(rf"Compiling entry function '([^']*{kernel}[^']*)'.*?Used (\d+) registers", ptxas_log, re.S)
-    if not found:
-        raise RuntimeError(f"{os.path.basename(src)}: no ptxas register report for {kernel}")
+    found = []
+    for kernel in REG_SPLIT_SOURCES[os.path.basename(src)]:
+        hits = re.findall(rf"Compiling entry function '([^']*\d{kernel}[IE][^']*)'.*?Used (\d+) registers", ptxas_log, re.S)
+        if not hits:
+            raise RuntimeError(f"{os.path.basename(src)}: no ptxas register report for {kernel}")
+        found += hits
     for name, regs in found:
         regs = int(regs)
         low_threads = 128

@@ -222,7 +222,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         pp.out = static_cast<__nv_bfloat16 *>(out);
         pp.tiles = reinterpret_cast<const PrefillTile *>(tb + tl.tiles);
         pp.cta_start = reinterpret_cast<const int32_t *>(tb + tl.cta_start);
-        pp.num_ctas = plan->num_prefill_ctas;
+        pp.pair = plan->prefill_pair ? 1 : 0;
+        pp.num_ctas = plan->prefill_pair ? plan->num_prefill_ctas / 2 : plan->num_prefill_ctas;
         pp.stages = reinterpret_cast<const StageTile *>(tb + tl.stages);
         pp.staged = ws + w.staged;
         pp.num_stages = plan->num_stages;

@@ -64,7 +64,8 @@ struct PrefillParams {
     float2 *partial_ml;       // [pieces][G]: (max in log2 units, sum)
     uint32_t *status;
     int num_tiles;
-    int num_ctas;
+    int num_ctas;   // persistent CTAs, or with `pair` clusters of two CTAs
+    int pair;       // every tile's two heads on a cluster of two CTAs (one head each)
     int num_stages;
     int num_tokens;  // rows of q (extent of its TMA descriptor)
     int num_blocks;  // blocks of the pool (extent of the cache descriptors)

@@ -64,6 +64,10 @@ constexpr int64_t kRowCostBlocks = 8;
 // GPU (~3.5 us with all SMs); the decode kernel streams ~66 GB/s per SM
 // up to ~6.1 TB/s of HBM bandwidth (reached from ~92 SMs on).
 constexpr double kPrefillStepUs = 2.9;
+// The same step of a two-head tile on a cluster of two SMs (the pair kernel:
+// one head per SM, 2-SM MMAs), in microseconds of the cluster; measured on
+// B200 at ~1.22 on long chunks beside the decode kernel.
+constexpr double kPairStepUs = 1.25;
 constexpr double kDecodeBytesPerUsPerSm = 66e3;
 constexpr double kHbmBytesPerUs = 6.1e6;
 constexpr int kMinSideSms = 8;  // fewest SMs either kernel is given when they share the GPU
@@ -118,16 +122,16 @@ std::vector<PrefixGroup> find_prefix_groups(const int32_t *h_cu, const int32_t *
 
 // SMs for the prefill kernel when it runs beside the decode kernel, or 0 when
 // running them one after the other is predicted to be as fast.
-int overlap_split(int num_sms, int64_t prefill_steps, int64_t decode_bytes) {
+int overlap_split(int num_sms, int64_t prefill_steps, int64_t decode_bytes, double step_sm_us) {
     if (prefill_steps <= 0 || decode_bytes <= 0 || num_sms < 2 * kMinSideSms) return 0;
     auto decode_us = [&](int sms) {
         return (double)decode_bytes / std::min(kHbmBytesPerUs, sms * kDecodeBytesPerUsPerSm);
     };
-    const double serial = prefill_steps * kPrefillStepUs / num_sms + decode_us(num_sms);
+    const double serial = prefill_steps * step_sm_us / num_sms + decode_us(num_sms);
     double best = serial;
     int best_p = 0;
     for (int s = kMinSideSms; s <= num_sms - kMinSideSms; ++s) {
-        const double t = std::max(prefill_steps * kPrefillStepUs / s, decode_us(num_sms - s));
+        const double t = std::max(prefill_steps * step_sm_us / s, decode_us(num_sms - s));
         if (t < best) {
             best = t;
             best_p = s;
@@ -153,7 +157,7 @@ struct CascadeChoice {
 };
 
 CascadeChoice choose_cascade(int num_sms, int G, int Hkv, const std::vector<PrefixGroup> &groups,
-                             int64_t other_total, int64_t other_max, int64_t decode_cost_bytes) {
+                             int64_t other_total, int64_t other_max, int64_t decode_cost_bytes, bool pair) {
     CascadeChoice best;
     double best_us = 1e30;
     int nt_min = INT32_MAX;
@@ -169,10 +173,13 @@ CascadeChoice choose_cascade(int num_sms, int G, int Hkv, const std::vector<Pref
             tiles += cdiv(g.nseg, pa::kPrefillTileM) * Hkv * cdiv(G, 2) * sp;
             cost = std::max<int64_t>(cost, cdiv(nt, sp) + kPrefixTileOverheadSteps);
         }
+        // s SMs hold s persistent CTAs, or s / 2 clusters with the pair kernel
         auto prefill_us = [&](int s) {
-            double units = (double)cdiv(tiles, s) * cost;
-            if (other_total > 0) units += (double)other_total / s + (double)other_max;
-            return units * kPrefillStepUs;
+            const int slots = pair ? s / 2 : s;
+            if (slots < 1) return 1e30;
+            double units = (double)cdiv(tiles, slots) * cost;
+            if (other_total > 0) units += (double)other_total / slots + (double)other_max;
+            return units * (pair ? kPairStepUs : kPrefillStepUs);
         };
         // one after the other, on every SM
         double t = prefill_us(num_sms) + decode_us(num_sms);
@@ -180,7 +187,7 @@ CascadeChoice choose_cascade(int num_sms, int G, int Hkv, const std::vector<Pref
             best_us = t;
             best = {sp, 0};
         }
-        for (int s = kMinSideSms; s <= num_sms - kMinSideSms; ++s) {
+        for (int s = kMinSideSms; s <= num_sms - kMinSideSms; s += pair ? 2 : 1) {
             t = std::max(prefill_us(s), decode_us(num_sms - s));
             if (t < best_us) {
                 best_us = t;
@@ -403,6 +410,11 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     // query-head pair and key split, with the splits (and the SMs the
     // prefill kernel gets beside the decode kernel) chosen by
     // choose_cascade.
+    // The pair kernel takes a tile's two heads on a cluster of two SMs; it
+    // serves plans whose every tile has two heads (an even group size) at
+    // head_dim 128.
+    bool pair = pa::prefill_kernel_available() && G % 2 == 0 && d.head_dim == 128;
+    for (const pa::PrefillTile &t : tiles) pair = pair && t.num_heads == 2;
     CascadeChoice cascade_choice;
     if (!groups.empty()) {
         int64_t other_total = 0, other_max = 0;
@@ -414,7 +426,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         for (const pa::DecodeRow &r : rows)
             decode_cost_blocks += cdiv(r.n_keys, pa::kBlockSize) - r.first_block + kRowCostBlocks;
         cascade_choice = choose_cascade(p->num_sms, G, Hkv, groups, other_total, other_max,
-                                        decode_cost_blocks * pa::kBlockSize * d.head_dim * 2 * 2);
+                                        decode_cost_blocks * pa::kBlockSize * d.head_dim * 2 * 2, pair);
     }
     for (size_t k = 0; k < groups.size(); ++k) {
         const PrefixGroup &gr = groups[k];
@@ -453,12 +465,16 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     // merging to a merge kernel after both.
     p->cascade = !groups.empty();
     p->num_prefix_groups = (int32_t)groups.size();
+    p->prefill_pair = pair && !tiles.empty();
     p->overlap_sms = groups.empty()
-                         ? overlap_split(p->num_sms, prefill_steps, decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2)
+                         ? overlap_split(p->num_sms, prefill_steps, decode_blocks_all * pa::kBlockSize * d.head_dim * 2 * 2,
+                                         p->prefill_pair ? 2 * kPairStepUs : kPrefillStepUs)
                          : cascade_choice.sms;
+    if (p->prefill_pair) p->overlap_sms &= ~1;  // whole SM pairs
     const int prefill_sms = p->overlap_sms > 0 ? p->overlap_sms : p->num_sms;
     const int decode_sms = p->num_sms - p->overlap_sms;
-    const int grid = (int)std::min<size_t>(tiles.size(), (size_t)prefill_sms);
+    // persistent CTAs, or with the pair kernel clusters of two, one per tile slot
+    const int grid = (int)std::min<size_t>(tiles.size(), (size_t)(p->prefill_pair ? prefill_sms / 2 : prefill_sms));
     std::vector<int32_t> cta_start(grid + 1, 0);
     if (grid > 0) {
         std::vector<std::vector<int32_t>> per(grid);
@@ -559,7 +575,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     p->decode_keys = 0;
     for (const pa::DecodeRow &r : rows) p->decode_keys += r.n_keys - (int64_t)r.first_block * pa::kBlockSize;
     p->num_tiles = (int32_t)tiles.size();
-    p->num_prefill_ctas = grid;
+    p->num_prefill_ctas = p->prefill_pair ? 2 * grid : grid;
     p->num_stages = (int32_t)stages.size();
 
     pa::TableLayout &t = p->tl;

@@ -145,6 +145,7 @@ struct pa_plan {
     // prefill part
     int32_t num_tiles = 0;
     int32_t num_prefill_ctas = 0;        // persistent prefill CTAs (one per SM at most)
+    bool prefill_pair = false;           // tiles run on clusters of two CTAs (num_prefill_ctas / 2 clusters)
     int32_t overlap_sms = 0;             // > 0: prefill runs on this many SMs beside the decode kernel
     bool cascade = false;                // shared-prefix tiles: the prefill kernel runs first
     int32_t num_prefix_groups = 0;

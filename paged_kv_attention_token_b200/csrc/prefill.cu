@@ -400,6 +400,7 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
 // {64, 1, 128}: one 64-dim slab of 128 tokens of one head, 128-byte swizzle.
 struct PrefillMaps {
     CUtensorMap q;
+    CUtensorMap out;  // the same shape over the output (pair kernel's stores)
 };
 
 // Gathers staged tile blockIdx.x (K for blockIdx.y = 0, V for 1) from the
@@ -740,6 +741,683 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Pair kernel (head_dim 128): one tile per cluster of two CTAs on two SMs.
+// The CTA of cluster rank r holds head A + r of the tile, and every product
+// runs as one MMA over both SMs (tcgen05 with cta_group::2, M = 256).
+//
+// The two-head kernel above keeps both heads of a tile in one SM's 512 TMEM
+// columns, so each head has a single S buffer and its loop S(j) -> softmax
+// -> PV(j) -> S(j + 1) is serial.  Here each SM holds one head: two S
+// buffers (256 columns) and O.  S(j + 2) is computed into the buffer P(j)
+// occupied, right after PV(j), so the softmax finds the next S ready.
+//
+// A 2-SM MMA takes the 256 rows of A from both CTAs (rows 0-127 from rank 0,
+// 128-255 from rank 1: the two heads' Q in shared memory, or their P in
+// TMEM), splits B by its N columns (rank r holds columns N/2 r ..
+// N/2 r + N/2 - 1) and writes each CTA's 128 rows of D into that CTA's TMEM.
+// So for S = Q K^T rank r loads keys 64 r .. 64 r + 63 of a K tile, and for
+// O += P V dims 64 r .. 64 r + 63 of a V tile: each K/V byte crosses from L2
+// into shared memory once per pair, and each SM's MMAs read half of B.  Per
+// 128-key step and SM that is 32 KB of loads and 64 KB of operand reads
+// beside the 1024 tensor cycles of the step's two products; a single SM
+// holding both heads moves 256 KB per two such steps.
+//
+// Rank 0 issues every MMA (one thread) and owns the barriers that gate them:
+// a K/V stage or Q is ready once a forwarding thread in each CTA has seen
+// that CTA's copy land and arrived on rank 0's barrier; P and the release of
+// O wait for the softmax warps of both CTAs (remote arrivals).  Every commit
+// arrives in both CTAs (tcgen05.commit cta_group::2 with cluster multicast),
+// so each CTA's loader, softmax warps and epilogue wait on barriers of their
+// own.  No TMA or bulk load uses cluster multicast.
+//
+// Eight softmax warps per CTA split every query row into two halves of 64
+// keys (warps 4-7 and 8-11 share TMEM lanes and exchange the half-row maxima
+// and sums through shared memory).
+// ---------------------------------------------------------------------------
+struct PairCfg {
+    static constexpr int D = 128;
+    static constexpr int kThreads = 384;
+    static constexpr int kSoftHi = 8;                      // warps 4-7: keys 0-63 of a step, warps 8-11: 64-127
+    static constexpr int kTileBytes = 128 * D * 2;         // a staged K or V tile (two 64-dim slabs of 16 KB)
+    static constexpr int kQBytes = 128 * D * 2;            // Q of this CTA's head
+    static constexpr int kKBytes = 64 * D * 2;             // this CTA's 64 keys of a K tile (8 KB of each slab)
+    static constexpr int kVBytes = 128 * 64 * 2;           // this CTA's 64 dims of a V tile (one slab)
+    static constexpr int kKStages = 5;
+    static constexpr int kVStages = 4;
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQBytes;
+    static constexpr int kVOff = kKOff + kKStages * kKBytes;
+    static constexpr int kXchOff = kVOff + kVStages * kVBytes;  // float [2 slots][2 halves][128 rows]
+    static constexpr int kOutOff = kXchOff + 2 * 2 * 128 * 4;   // bf16 output tile: two 64-dim slabs, 128-byte swizzle
+    static constexpr int kBarOff = kOutOff + 128 * D * 2;
+    // mbarriers.  "land": this CTA's copy arrived (its own loads' bytes);
+    // "ready": both CTAs' copies arrived (used in rank 0, one arrival per
+    // CTA); "empty": the MMAs reading a stage completed (multicast commit).
+    static constexpr int kBarQLand = 0, kBarQReady = 1, kBarQEmpty = 2;
+    static constexpr int kBarKLand = 3;
+    static constexpr int kBarKReady = kBarKLand + kKStages;
+    static constexpr int kBarKEmpty = kBarKReady + kKStages;
+    static constexpr int kBarVLand = kBarKEmpty + kKStages;
+    static constexpr int kBarVReady = kBarVLand + kVStages;
+    static constexpr int kBarVEmpty = kBarVReady + kVStages;
+    static constexpr int kSBufs = 2;                       // S buffers in TMEM
+    static constexpr int kBarS = kBarVEmpty + kVStages;    // [kSBufs]: S of the step in TMEM buffer b
+    static constexpr int kBarP = kBarS + kSBufs;           // [kSBufs][2]: P of half h in buffer b, both CTAs (rank 0)
+    static constexpr int kBarPV = kBarP + 2 * kSBufs;      // [2]: the PV product of half h completed
+    static constexpr int kBarO = kBarPV + 2;               // the tile's last PV products completed
+    static constexpr int kBarOFree = kBarO + 1;            // both CTAs read O (rank 0)
+    static constexpr int kBarDrain = kBarOFree + 1;        // every MMA issued completed
+    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+    static constexpr int kUsed = kTmemSlotOff + 16;
+    static constexpr int kSmemBytes = kUsed + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
+    static constexpr uint32_t kTmemCols = 512;
+    // S buffers at 0 and 128; the accumulators O_0 (keys 0-63 of every
+    // step) at 256 and O_1 (keys 64-127) at 384
+    static constexpr uint32_t kS = 0, kO = 256;
+    static constexpr int kLaunchRegs = 168;
+    static constexpr int kRegsLow = 104;
+    static constexpr int kRegsHigh = 200;
+    static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * kLaunchRegs, "register split");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrival on an mbarrier of any CTA of the cluster (shared::cluster address),
+// with the default semantics (release at CTA scope).  Measured on B200, an
+// arrival with .release.cluster costs its thread ~1000 cycles; the data it
+// hands over is TMEM (completed by tcgen05.wait::st and ordered by
+// tcgen05.fence::before_thread_sync) or the other CTA's own copies, whose
+// completion the arriving thread observed on its mbarrier.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// TMEM allocation shared by the two CTAs (one warp of each executes it).
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t smem_dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// One lane of the (converged) warp: 1 there, 0 elsewhere.
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r));
+    return r;
+}
+// The MMA helpers below are executed by a whole warp with the operands
+// warp-uniform; only the lane with `issue` != 0 issues the instruction.
+// 2-SM MMA, A and B in shared memory (same offsets in both CTAs).
+__device__ __forceinline__ void umma_pair_ss(uint32_t issue, uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %6, 0;\n\t"
+        "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(issue));
+}
+// 2-SM MMA, A in TMEM (each CTA's 128 rows), B in shared memory.
+__device__ __forceinline__ void umma_pair_ts(uint32_t issue, uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %6, 0;\n\t"
+        "@q tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(issue));
+}
+// Arrives once on `bar` in both CTAs when every MMA issued so far is
+// complete (issued by the lane with `issue` != 0).
+__device__ __forceinline__ void umma_commit_pair(uint32_t issue, uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %2, 0;\n\t"
+        "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3), "r"(issue)
+        : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// 3-D tiled TMA store (no multicast) of a shared-memory box, tracked in this
+// thread's bulk async-group; c0 must be a multiple of 8 bf16 elements.
+__device__ __forceinline__ void tma_store_3d(const void *map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the shared memory of this thread's bulk stores has been read.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Softmax of one tile for this thread's half row: keys 64 half .. + 63 of
+// every step, as an online softmax of its own (running max m, sum l and the
+// accumulator O_half in TMEM), so that the two warps on an SM sub-partition
+// never wait for each other within a tile.  The halves combine at the end:
+// with M = max(m0, m1), O = (O_0 2^(m0 - M) + O_1 2^(m1 - M)) / (l0 2^(m0 - M)
+// + l1 2^(m1 - M)).  g counts the steps over the CTA's tiles, (sb, sph) the
+// TMEM buffer of the next step and the phase of its barriers, k the tiles,
+// e the end-of-tile exchanges with the partner thread (same row, other half).
+// p_full0 and o_free0 are rank 0's barriers (shared::cluster addresses);
+// out_stage is the shared-memory staging of the output tile, stored through
+// out_map.
+__device__ __forceinline__ void pair_softmax_tile(const PrefillParams &p, const PrefillTile &tile, uint32_t trow,
+                                                  int half, float *xch, uint64_t *s_full, uint32_t p_full0,
+                                                  uint64_t *pv_done, uint64_t *o_done, uint32_t o_free0, uint32_t &g,
+                                                  uint32_t &sb, uint32_t &sph, uint32_t k, const CUtensorMap *out_map,
+                                                  uint32_t out_stage, uint32_t &e, int t, int quarter, int q_rows,
+                                                  int pos, int first_pos, int tok0, int head, int hl, bool &err) {
+    using C = PairCfg;
+    constexpr int D = C::D;
+    constexpr int kHalfO = D / 2;  // output columns of this thread
+    const uint32_t o_mine = C::kO + 128 * half;
+    float m = -INFINITY, l = 0.f;
+    const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
+    auto exchange = [&](float v) {  // the partner thread's value of v
+        float *slot = xch + (e & 1u) * 256;
+        slot[half * 128 + t] = v;
+        named_sync(1 + quarter, 64);
+        const float o = slot[(half ^ 1) * 128 + t];
+        ++e;
+        return o;
+    };
+    for (int j = 0; j < tile.n_kv_tiles; ++j, ++g) {
+        const uint32_t b = sb;
+        if (!err && !mbar_wait(&s_full[b], sph, p.wait_limit)) err = true;
+        if (++sb == C::kSBufs) { sb = 0; sph ^= 1u; }
+        tc_fence_after();
+        const int kbase = 128 * (tile.kv_tile0 + j) + 64 * half;  // first key of this half step
+        const bool masked = kbase + 63 > first_pos;
+        // S of this half in columns 64 half .. + 63; its P (bf16 pairs) goes
+        // to columns 64 half .. + 31, which no other thread reads
+        const uint32_t s_col = C::kS + 128 * b + 64 * half;
+        uint32_t s0[32], s1[32];
+        tmem_ld32(trow + s_col, s0);
+        tmem_ld32(trow + s_col + 32, s1);
+        tmem_ld_wait();
+        const float mx =
+            fmaxf(chunk_max(s0, masked, kbase, pos), chunk_max(s1, masked, kbase + 32, pos)) * p.scale_log2;
+        float alpha = 1.f;
+        const bool rescale = mx > m + kPrefillRescaleThreshold;
+        if (rescale) {
+            alpha = fast_exp2(m - mx);
+            m = mx;
+        }
+        const uint64_t nm2 = f2(-m, -m);
+        uint32_t pk0[16], pk1[16];
+        chunk_exp(s0, pk0, scale2, nm2, masked, kbase, pos);
+        tmem_st16(trow + s_col, pk0);
+        chunk_exp(s1, pk1, scale2, nm2, masked, kbase + 32, pos);
+        tmem_st16(trow + s_col + 16, pk1);
+        // O_half is rescaled after the previous step's PV product for this
+        // half completed and before this step's P is handed over
+        if (j > 0 && __any_sync(kFullMask, rescale)) {
+            if (!err && !mbar_wait(&pv_done[half], (g - 1) & 1u, p.wait_limit)) err = true;
+            tc_fence_after();
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {
+                uint32_t o[32];
+                tmem_ld32(trow + o_mine + 32 * i, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                tmem_st32(trow + o_mine + 32 * i, o);
+            }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive_remote(p_full0 + 8 * (2 * b + half));
+        // the sum of the rounded P values the PV product uses
+        regs_after(pk0);
+        regs_after(pk1);
+        float l0, l1;
+        f2_split(f2_add(chunk_sum(pk0), chunk_sum(pk1)), l0, l1);
+        l = l * alpha + (l0 + l1);
+    }
+    if (!err && !mbar_wait(o_done, k & 1u, p.wait_limit)) err = true;
+    tc_fence_after();
+    // both halves of the row: the same maximum M and sum L in both threads
+    const float m_o = exchange(m), l_o = exchange(l);
+    const float mm = fmaxf(m, m_o);
+    const float c_me = fast_exp2(m - mm), c_o = fast_exp2(m_o - mm);
+    const float lsum = l * c_me + l_o * c_o;
+    // output columns kHalfO half .. + kHalfO - 1 from both accumulators
+    const uint32_t o_other = C::kO + 128 * (half ^ 1);
+    uint32_t o[kHalfO / 32][32];
+#pragma unroll
+    for (int i = 0; i < kHalfO / 32; ++i) {
+        uint32_t x[32];
+        tmem_ld32(trow + o_mine + kHalfO * half + 32 * i, o[i]);
+        tmem_ld32(trow + o_other + kHalfO * half + 32 * i, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+            o[i][c] = __float_as_uint(__uint_as_float(o[i][c]) * c_me + __uint_as_float(x[c]) * c_o);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive_remote(o_free0);
+    if (tile.row_base >= 0) {
+        if (t < q_rows) {
+            const int G = p.group;
+            const int r = tile.row_base + t * p.num_kv_heads;
+            const int slot = p.combine[p.rows[r].combine].piece_base + tile.piece;
+            float *po = p.partial_o + ((size_t)slot * G + hl) * D + kHalfO * half;
+#pragma unroll
+            for (int i = 0; i < kHalfO / 32; ++i)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    reinterpret_cast<float4 *>(po + 32 * i)[c] =
+                        make_float4(__uint_as_float(o[i][4 * c]), __uint_as_float(o[i][4 * c + 1]),
+                                    __uint_as_float(o[i][4 * c + 2]), __uint_as_float(o[i][4 * c + 3]));
+            if (half == 0) p.partial_ml[(size_t)slot * G + hl] = make_float2(mm, lsum);
+        }
+        return;
+    }
+    const float inv = 1.f / lsum;
+    if (q_rows == 128) {
+        // A full tile: the half rows go through shared memory (the 128-byte
+        // swizzled box of the output's tensor map) and leave as one TMA
+        // store per half, so that the rows' scattered 16-byte pieces become
+        // whole lines and the warps need not wait for them.
+        const uint32_t slab = out_stage + half * 16384;
+        const bool issuer = (threadIdx.x & 127) == 0;
+        if (issuer) bulk_wait_read();  // the previous tile's store has read the slab
+        named_sync(5 + half, 128);
+#pragma unroll
+        for (int i = 0; i < kHalfO / 32; ++i) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[i][8 * c + 0]) * inv, __uint_as_float(o[i][8 * c + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(o[i][8 * c + 2]) * inv, __uint_as_float(o[i][8 * c + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(o[i][8 * c + 4]) * inv, __uint_as_float(o[i][8 * c + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(o[i][8 * c + 6]) * inv, __uint_as_float(o[i][8 * c + 7]) * inv);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(swz128(slab, t, 4 * i + c)), "r"(w.x),
+                             "r"(w.y), "r"(w.z), "r"(w.w)
+                             : "memory");
+            }
+        }
+        fence_proxy_async_smem();
+        named_sync(5 + half, 128);
+        if (issuer) tma_store_3d(out_map, slab, 64 * half, head, tok0);
+        return;
+    }
+    if (t < q_rows) {
+        __nv_bfloat16 *orow = p.out + ((size_t)(tok0 + t) * p.num_q_heads + head) * D + kHalfO * half;
+#pragma unroll
+        for (int i = 0; i < kHalfO / 32; ++i) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[i][8 * c + 0]) * inv, __uint_as_float(o[i][8 * c + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(o[i][8 * c + 2]) * inv, __uint_as_float(o[i][8 * c + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(o[i][8 * c + 4]) * inv, __uint_as_float(o[i][8 * c + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(o[i][8 * c + 6]) * inv, __uint_as_float(o[i][8 * c + 7]) * inv);
+                st16(orow + 32 * i + 8 * c, w);
+            }
+        }
+    }
+}
+
+// Cluster c (CTAs 2c and 2c + 1) works through tiles [cta_start[c],
+// cta_start[c + 1]); every tile has two heads.  Both CTAs run the same tile
+// list, so they take the same K/V stages in the same order and both reach
+// every cluster barrier.
+__global__ void __launch_bounds__(384, 1)
+    prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps maps) {
+    using C = PairCfg;
+    constexpr int D = C::D;
+    extern __shared__ uint8_t smem_raw[];
+    // the same 1024-aligned offset in both CTAs: the 2-SM MMAs read both
+    // CTAs' operands through one descriptor
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sQ = smem_u32(smem + C::kQOff);
+    const uint32_t sK = smem_u32(smem + C::kKOff);
+    const uint32_t sV = smem_u32(smem + C::kVOff);
+    float *xch = reinterpret_cast<float *>(smem + C::kXchOff);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *q_land = bars + C::kBarQLand, *q_ready = bars + C::kBarQReady, *q_empty = bars + C::kBarQEmpty;
+    uint64_t *k_land = bars + C::kBarKLand, *k_ready = bars + C::kBarKReady, *k_empty = bars + C::kBarKEmpty;
+    uint64_t *v_land = bars + C::kBarVLand, *v_ready = bars + C::kBarVReady, *v_empty = bars + C::kBarVEmpty;
+    uint64_t *s_full = bars + C::kBarS, *p_full = bars + C::kBarP, *pv_done = bars + C::kBarPV;
+    uint64_t *o_done = bars + C::kBarO, *o_free = bars + C::kBarOFree, *drain = bars + C::kBarDrain;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kTmemSlotOff);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank();
+    const int cl = blockIdx.x >> 1;
+    // (the launch has exactly num_ctas clusters; a cluster with no tiles
+    // still takes every cluster barrier below)
+    const int t_begin = p.cta_start[cl], t_end = p.cta_start[cl + 1];
+
+    if (tid == 0) {
+        mbar_init(q_land, 1);
+        mbar_init(q_ready, 2);  // one forwarder per CTA
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < C::kKStages; ++s) {
+            mbar_init(&k_land[s], 1);
+            mbar_init(&k_ready[s], 2);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < C::kVStages; ++s) {
+            mbar_init(&v_land[s], 1);
+            mbar_init(&v_ready[s], 2);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int b = 0; b < C::kSBufs; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[2 * b], 8);  // one arrival per softmax warp of the half, both CTAs
+            mbar_init(&p_full[2 * b + 1], 8);
+        }
+        mbar_init(&pv_done[0], 1);
+        mbar_init(&pv_done[1], 1);
+        mbar_init(o_done, 1);
+        mbar_init(o_free, 16);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // both CTAs' barriers are initialised before either touches the other's
+    cluster_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool err = false;
+    // rank 0's copy of a barrier of this CTA's layout
+    auto at_rank0 = [](uint64_t *bar) { return peer_addr(smem_u32(bar), 0); };
+
+    if (warp < 4) {
+        warpgroup_reg_dealloc<C::kRegsLow>();
+        if (warp == 0 && rank == 0) {
+            // ------------------------------------------------ MMA issuer (rank 0, warp 0; one lane issues)
+            //   S(j) = Q K_j^T (M 256, N 128, K D) into TMEM buffer j % 2,
+            //   PV_h(j): O_h += P_h(j) V_h,j (M 256, N D, K 64: keys
+            //   64 h .. 64 h + 63 of the step, A = P from TMEM),
+            // issued S(0) S(1) | PV_0(0) PV_1(0) S(2) | PV_0(1) PV_1(1) S(3)
+            // | ...: each half's PV goes as soon as that half's P is there,
+            // and S(j + 2) reuses the buffer both PV(j) have just read
+            // (tcgen05 MMAs of one thread run in issue order).
+            const uint32_t me = elect_one();
+            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(256, 128, false, false);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(256, D, false, true);
+            const uint64_t dQ = umma_desc_sw128(sQ, 16, 1024);
+            const uint64_t dK = umma_desc_sw128(sK, 16, 1024), dV = umma_desc_sw128(sV, 16384, 1024);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                if (!err && !mbar_wait(bar, parity, p.wait_limit)) err = true;
+            };
+            int vs = 0, ks = 0;
+            uint32_t vph = 0, kph = 0;
+            uint32_t k = 0;                           // tiles so far
+            uint32_t sb = 0, pb = 0, pph = 0;         // buffer of the next S, of the next P and its phase
+            for (int ti = t_begin; ti < t_end; ++ti) {
+                const PrefillTile tile = p.tiles[ti];
+                const int n = tile.n_kv_tiles;
+                int s_issued = 0;
+                auto issue_s = [&]() {
+                    wait(&k_ready[ks], kph);
+                    tc_fence_after();
+                    const uint64_t dk = dK + ks * (uint32_t)(C::kKBytes >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // 16 dims = 32 bytes along a 128-byte row; 64-dim slabs
+                        // 16 KB apart in Q, 8 KB apart in this CTA's K half
+                        const uint32_t q_off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                        const uint32_t k_off = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                        umma_pair_ss(me, tmem + C::kS + 128 * sb, dQ + q_off, dk + k_off, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit_pair(me, &s_full[sb]);
+                    umma_commit_pair(me, &k_empty[ks]);
+                    if (++ks == C::kKStages) { ks = 0; kph ^= 1u; }
+                    if (++sb == C::kSBufs) sb = 0;
+                    // the tile's last S product releases Q
+                    if (++s_issued == n) umma_commit_pair(me, q_empty);
+                };
+                wait(q_ready, (uint32_t)(ti - t_begin) & 1u);
+                for (int j = 0; j < C::kSBufs && j < n; ++j) issue_s();
+                for (int j = 0; j < n; ++j) {
+                    const uint64_t dv = dV + vs * (uint32_t)(C::kVBytes >> 4);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        wait(&p_full[2 * pb + h], pph);
+                        if (h == 0) {
+                            if (j == 0 && k > 0) wait(o_free, (k - 1) & 1u);
+                            wait(&v_ready[vs], vph);
+                        }
+                        tc_fence_after();
+                        // P_h: bf16 pairs in columns 64 h .. + 31 of the buffer;
+                        // V rows (keys) 64 h + 16 kk .. + 15, 128 bytes each
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_pair_ts(me, tmem + C::kO + 128 * h, tmem + C::kS + 128 * pb + 64 * h + 8 * kk,
+                                         dv + (((64 * h + 16 * kk) * 128) >> 4), idesc_pv, kk > 0 || j > 0 ? 1u : 0u);
+                        umma_commit_pair(me, &pv_done[h]);
+                    }
+                    if (j + 1 == n) umma_commit_pair(me, o_done);
+                    umma_commit_pair(me, &v_empty[vs]);
+                    if (++vs == C::kVStages) { vs = 0; vph ^= 1u; }
+                    if (++pb == C::kSBufs) { pb = 0; pph ^= 1u; }
+                    if (j + C::kSBufs < n) issue_s();
+                }
+                ++k;
+            }
+            umma_commit_pair(me, drain);
+            if (!mbar_wait(drain, 0, p.wait_limit)) err = true;
+        } else if (warp == 0 && lane == 0) {
+            // rank 1: the last commit (and with it every earlier one) has
+            // arrived here before the CTA may end
+            if (!mbar_wait(drain, 0, p.wait_limit)) err = true;
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------------------------ loads (both CTAs)
+            // In the order the MMAs consume them, per tile: Q, K0 K1 K2, V0 K3
+            // V1 K4 ...  A stage is reloaded once the MMAs that read it (in both
+            // CTAs) completed.
+            int vs = 0, ks = 0;
+            uint32_t vuse = 0, kuse = 0;
+            for (int ti = t_begin; ti < t_end; ++ti) {
+                const PrefillTile tile = p.tiles[ti];
+                const int n = tile.n_kv_tiles;
+                const int tok0 = tile.row_base >= 0 ? tile.q_start : p.cu_seqlens_q[tile.seq] + tile.q_start;
+                if (ti > t_begin && !err &&
+                    !mbar_wait(q_empty, (uint32_t)(ti - t_begin - 1) & 1u, p.wait_limit))
+                    err = true;
+                mbar_arrive_expect_tx(q_land, C::kQBytes);
+#pragma unroll
+                for (int s = 0; s < D / 64; ++s)
+                    tma_load_3d(sQ + s * 16384, &maps.q, q_land, 64 * s, tile.head + (int)rank, tok0);
+                const uint8_t *kv = p.staged + (size_t)(tile.kv_base + tile.kv_tile0) * 2 * C::kTileBytes;
+                auto load_k = [&](const uint8_t *kt) {
+                    if (kuse >= (uint32_t)C::kKStages && !err &&
+                        !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1u, p.wait_limit))
+                        err = true;
+                    mbar_arrive_expect_tx(&k_land[ks], C::kKBytes);
+                    // keys 64 rank .. + 63 of both 64-dim slabs
+#pragma unroll
+                    for (int s = 0; s < D / 64; ++s)
+                        bulk_load(sK + ks * C::kKBytes + s * 8192, kt + s * 16384 + rank * 8192, 8192, &k_land[ks]);
+                    ++kuse;
+                    if (++ks == C::kKStages) ks = 0;
+                };
+                auto load_v = [&](const uint8_t *vt) {
+                    if (vuse >= (uint32_t)C::kVStages && !err &&
+                        !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1u, p.wait_limit))
+                        err = true;
+                    mbar_arrive_expect_tx(&v_land[vs], C::kVBytes);
+                    bulk_load(sV + vs * C::kVBytes, vt + rank * 16384, C::kVBytes, &v_land[vs]);  // dims 64 rank ..
+                    ++vuse;
+                    if (++vs == C::kVStages) vs = 0;
+                };
+                for (int j = 0; j < C::kSBufs && j < n; ++j) load_k(kv + (size_t)j * 2 * C::kTileBytes);
+                for (int j = 0; j < n; ++j) {
+                    load_v(kv + ((size_t)j * 2 + 1) * C::kTileBytes);
+                    if (j + C::kSBufs < n) load_k(kv + (size_t)(j + C::kSBufs) * 2 * C::kTileBytes);
+                }
+            }
+        } else if (warp == 2 && lane == 0) {
+            // ------------------------------------------------ forwarder (both CTAs)
+            // Walks the loads in the loader's order; once this CTA's copy has
+            // landed it arrives on rank 0's ready barrier.  Having waited for
+            // every landing, it also guarantees that no copy into this CTA is
+            // in flight when the CTA ends.
+            int vs = 0, ks = 0;
+            uint32_t vuse = 0, kuse = 0;
+            auto fwd = [&](uint64_t *land, uint64_t *ready, uint32_t parity) {
+                if (!mbar_wait(land, parity, p.wait_limit)) err = true;
+                mbar_arrive_remote(at_rank0(ready));
+            };
+            auto fwd_k = [&]() {
+                fwd(&k_land[ks], &k_ready[ks], (kuse / C::kKStages) & 1u);
+                ++kuse;
+                if (++ks == C::kKStages) ks = 0;
+            };
+            auto fwd_v = [&]() {
+                fwd(&v_land[vs], &v_ready[vs], (vuse / C::kVStages) & 1u);
+                ++vuse;
+                if (++vs == C::kVStages) vs = 0;
+            };
+            for (int ti = t_begin; ti < t_end; ++ti) {
+                const int n = p.tiles[ti].n_kv_tiles;
+                fwd(q_land, q_ready, (uint32_t)(ti - t_begin) & 1u);
+                for (int j = 0; j < C::kSBufs && j < n; ++j) fwd_k();
+                for (int j = 0; j < n; ++j) {
+                    fwd_v();
+                    if (j + C::kSBufs < n) fwd_k();
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax warps (both CTAs)
+        warpgroup_reg_alloc<C::kRegsHigh>();
+        const int half = warp < C::kSoftHi ? 0 : 1;
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t p_full0 = at_rank0(p_full), o_free0 = at_rank0(o_free);
+        uint32_t g = 0, sb = 0, sph = 0, k = 0, e = 0;
+        // a tile's rows; the next tile's are read from global memory while
+        // the current one is worked on
+        struct Rows {
+            PrefillTile tile;
+            int tok0, q_rows, first_pos, pos;
+        };
+        auto rows_of = [&](int ti) {
+            Rows r;
+            r.tile = p.tiles[ti];
+            if (r.tile.row_base >= 0) {
+                r.tok0 = r.tile.q_start;
+                r.q_rows = r.tile.q_rows;
+                r.first_pos = r.tile.key_limit - 1;
+                r.pos = t < r.q_rows ? r.first_pos : 0;
+            } else {
+                const int seq = r.tile.seq, q0 = r.tile.q_start;
+                const int c0 = p.cu_seqlens_q[seq], c1 = p.cu_seqlens_q[seq + 1];
+                const int n = p.seq_lens[seq];
+                r.tok0 = c0 + q0;
+                r.q_rows = min(128, c1 - c0 - q0);
+                r.first_pos = n - (c1 - c0) + q0;
+                r.pos = t < r.q_rows ? r.first_pos + t : 0;
+            }
+            return r;
+        };
+        Rows cur = rows_of(t_begin < t_end ? t_begin : 0);
+        for (int ti = t_begin; ti < t_end; ++ti) {
+            const Rows nxt = rows_of(ti + 1 < t_end ? ti + 1 : ti);
+            const int head = cur.tile.head + (int)rank;
+            pair_softmax_tile(p, cur.tile, trow, half, xch, s_full, p_full0, pv_done, o_done, o_free0, g, sb, sph, k,
+                              &maps.out, smem_u32(smem + C::kOutOff), e, t, quarter, cur.q_rows, cur.pos,
+                              cur.first_pos, cur.tok0, head, head % p.group, err);
+            ++k;
+            cur = nxt;
+        }
+        // the output stores have read their shared memory before the CTA ends
+        if ((threadIdx.x & 127) == 0) bulk_wait_all();
+    }
+    if (err) atomicOr(p.status, kStatusWaitTimeout);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // rank 0 saw its last MMA complete, and each CTA its own copies land,
+    // before getting here: neither CTA frees TMEM or ends while the other's
+    // MMAs, copies or arrivals may still touch it
+    cluster_sync();
+    if (warp == 0) tmem_dealloc_pair(tmem, C::kTmemCols);
+}
+
+cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
+    using C = PairCfg;
+    constexpr int D = C::D;
+    EncodeFn enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    PrefillMaps maps;
+    const cuuint64_t dims[3] = {D, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.num_tokens};
+    const cuuint64_t strides[2] = {D * 2ull, (cuuint64_t)p.num_q_heads * D * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if (!encode_bf16(enc, &maps.q, p.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode_bf16(enc, &maps.out, p.out, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_relaxed) & bit)) {
+        cudaError_t e =
+            cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_relaxed);
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * p.num_ctas);  // num_ctas counts clusters here
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_pair_kernel, p, maps);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 }  // namespace
 
 bool prefill_kernel_available() { return true; }
@@ -755,6 +1433,7 @@ cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stre
 
 cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream) {
     if (p.num_tiles == 0) return cudaSuccess;
+    if (p.pair) return head_dim == 128 ? launch_prefill_pair(p, stream) : cudaErrorInvalidValue;
     return head_dim == 64 ? launch_prefill_t<64>(p, stream) : launch_prefill_t<128>(p, stream);
 }
 
