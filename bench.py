@@ -449,20 +449,21 @@ def run_ours(args):
                            "traffic": profiled_traffic("decode_kernel", args.workload, src_hash),
                            "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash}
     # when the plan runs the prefill kernel beside the decode kernel, it has
-    # num_prefill_ctas of the SMs: its peak is that share of the GPU's
-    side_by_side = bool(info["num_decode_units"] and info["num_prefill_tiles"]
-                        and info["num_prefill_ctas"] < info["num_sms"])
-    sm_share = info["num_prefill_ctas"] / info["num_sms"] if side_by_side else 1.0
+    # overlap_sms of the SMs: its peak is that share of the GPU's
+    side_by_side = bool(info["num_decode_units"] and info["num_prefill_tiles"] and info["overlap_sms"] > 0)
+    sm_share = info["overlap_sms"] / info["num_sms"] if side_by_side else 1.0
+    # head_dim 128 with an even group runs on the pair kernel (2-SM MMAs)
+    prefill_kernel = "prefill_pair_kernel" if info["prefill_pair"] else "prefill_kernel"
     if split["prefill_flops"] and prefill_ms > 0:
         tflops = split["prefill_flops"] / (prefill_ms * 1e-3) / 1e12
         pre_hash = kernel_source_hash(["prefill.cu", "common.cuh", "kernels.h", "plan.h"])
-        roofline_prefill = {"bound": "tensor", "kernel": "prefill_kernel", "achieved": tflops,
+        roofline_prefill = {"bound": "tensor", "kernel": prefill_kernel, "achieved": tflops,
                             "peak": peaks["bf16_tflops"] * sm_share,
                             "peak_kind": peak_kind + " (burst bf16" +
-                            (f", x {info['num_prefill_ctas']}/{info['num_sms']} SMs beside the decode kernel)"
+                            (f", x {info['overlap_sms']}/{info['num_sms']} SMs beside the decode kernel)"
                              if side_by_side else ")"),
                             "unit": "TFLOP/s", "frac": tflops / (peaks["bf16_tflops"] * sm_share),
-                            "traffic": profiled_traffic("prefill_kernel", args.workload, pre_hash),
+                            "traffic": profiled_traffic(prefill_kernel, args.workload, pre_hash),
                             "algorithmic_flops": split["prefill_flops"], "ms": prefill_ms,
                             "source_hash": pre_hash}
     # "roofline" is the dominant kernel's: the one with the longer device time

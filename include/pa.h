@@ -181,6 +181,12 @@ typedef struct {
                                      kernel attends (a row's keys, less a shared
                                      prefix the prefill kernel attends); unlike
                                      decode_kv_blocks, no padding of last blocks */
+    int32_t prefill_pair;         /* 1: the prefill tiles run on clusters of two
+                                     CTAs (num_prefill_ctas / 2 clusters, one
+                                     query head per CTA, 2-SM MMAs); 0: one CTA
+                                     per SM holds both heads of a tile */
+    int32_t overlap_sms;          /* > 0: SMs the prefill kernel runs on beside
+                                     the decode kernel; 0: one after the other */
 } pa_plan_info;
 int pa_plan_get_info(const pa_plan *plan, pa_plan_info *info);
 

@@ -68,7 +68,8 @@ class PlanInfo(ctypes.Structure):
                 ("table_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
                 ("num_staged_kv_tiles", ctypes.c_int32), ("num_prefill_ctas", ctypes.c_int32),
                 ("num_prefix_groups", ctypes.c_int32), ("attention_launches", ctypes.c_int32),
-                ("decode_kv_keys", ctypes.c_int64)]
+                ("decode_kv_keys", ctypes.c_int64), ("prefill_pair", ctypes.c_int32),
+                ("overlap_sms", ctypes.c_int32)]
 
     def as_dict(self):
         return {n: int(getattr(self, n)) for n, _ in self._fields_}

@@ -648,6 +648,8 @@ extern "C" int pa_plan_get_info(const pa_plan *p, pa_plan_info *info) {
     // prefill; the merge kernel when shared-prefix tiles run beside decode
     const bool side_by_side = p->overlap_sms > 0 && p->num_units > 0 && p->num_tiles > 0;
     info->decode_kv_keys = p->decode_keys;
+    info->prefill_pair = p->prefill_pair ? 1 : 0;
+    info->overlap_sms = p->overlap_sms;
     info->attention_launches = (p->num_units > 0 ? 1 : 0) + (p->num_tiles > 0 ? 1 : 0) +
                                (p->num_tiles > 0 && p->num_stages > 0 ? 1 : 0) +
                                (side_by_side && p->cascade && p->num_combine > 0 ? 1 : 0);

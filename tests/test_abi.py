@@ -94,12 +94,20 @@ def test_plan_invariants(lib, name):
     # every prefill segment are staged per kv head in 128-key tiles
     # (when decode rows exist too, the planner may give the prefill kernel a
     # share of the SMs to run beside the decode kernel, sized for the rest)
+    # (the pair kernel takes a tile's two heads on a cluster of two CTAs:
+    # head_dim 128, an even group, two CTAs per tile slot)
+    if info["prefill_pair"]:
+        assert lay.head_dim == 128 and G % 2 == 0 and info["num_prefill_ctas"] % 2 == 0
+    slots = info["num_sms"] // 2 if info["prefill_pair"] else info["num_sms"]
+    per_slot = 2 if info["prefill_pair"] else 1
     if info["num_decode_units"] == 0:
-        assert info["num_prefill_ctas"] == min(info["num_prefill_tiles"], info["num_sms"])
+        assert info["overlap_sms"] == 0
+        assert info["num_prefill_ctas"] == per_slot * min(info["num_prefill_tiles"], slots)
     else:
-        assert 0 <= info["num_prefill_ctas"] <= min(info["num_prefill_tiles"], info["num_sms"] - 8)
-        if info["num_prefill_ctas"] > 0:
-            assert info["num_decode_units"] <= (info["num_sms"] - info["num_prefill_ctas"]) * warps_per_sm
+        assert 0 <= info["num_prefill_ctas"] <= per_slot * min(info["num_prefill_tiles"], (info["num_sms"] - 8) // per_slot)
+        if info["overlap_sms"] > 0:
+            assert info["num_prefill_ctas"] <= info["overlap_sms"] <= info["num_sms"] - 8
+            assert info["num_decode_units"] <= (info["num_sms"] - info["overlap_sms"]) * warps_per_sm
     pre = ql > 16 if prefill_on_tensor_cores else np.zeros_like(ql, dtype=bool)
     staged = int(sum(-(-n // 128) for n in sl[pre])) * lay.num_kv_heads
     assert info["num_staged_kv_tiles"] == staged
