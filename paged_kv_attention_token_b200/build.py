@@ -50,26 +50,30 @@ def _stale(obj: str, src: str, newest_header: float) -> bool:
 # whose sum exceeds what the CTA was launched with would wait forever, so the
 # register count ptxas gives the kernel is checked against the split the
 # source assumes before the library is linked.
-REG_SPLIT_SOURCES = {"prefill.cu": ("prefill_kernel", "prefill_pair_kernel")}
+REG_SPLIT_SOURCES = {"prefill.cu": {"prefill_kernel": "PrefillCfg", "prefill_pair_kernel": "PairCfg"}}
 
 
 def check_register_split(src: str, ptxas_log: str) -> None:
     text = open(src).read()
-    want = {k: int(re.search(rf"{k} = (\d+);", text).group(1)) for k in ("kLaunchRegs", "kRegsLow", "kRegsHigh")}
-    threads = int(re.search(r"kThreads = (\d+);", text).group(1))
-    found = []
-    for kernel in REG_SPLIT_SOURCES[os.path.basename(src)]:
+    for kernel, cfg in REG_SPLIT_SOURCES[os.path.basename(src)].items():
+        # the kernel's constants, from the body of its configuration struct
+        m = re.search(rf"struct {cfg} {{(.*?)\n}};", text, re.S)
+        if not m:
+            raise RuntimeError(f"{os.path.basename(src)}: no struct {cfg}")
+        body = m.group(1)
+        want = {k: int(re.search(rf"{k} = (\d+);", body).group(1))
+                for k in ("kThreads", "kLaunchRegs", "kRegsLow", "kRegsHigh")}
         hits = re.findall(rf"Compiling entry function '([^']*\d{kernel}[IE][^']*)'.*?Used (\d+) registers", ptxas_log, re.S)
         if not hits:
             raise RuntimeError(f"{os.path.basename(src)}: no ptxas register report for {kernel}")
-        found += hits
-    for name, regs in found:
-        regs = int(regs)
-        low_threads = 128
-        need = low_threads * want["kRegsLow"] + (threads - low_threads) * want["kRegsHigh"]
-        if regs != want["kLaunchRegs"] or need > threads * regs:
-            raise RuntimeError(f"{name}: ptxas gives {regs} registers per thread at launch; the source assumes "
-                               f"{want['kLaunchRegs']} and a split needing {need} of {threads * regs}")
+        threads = want["kThreads"]
+        for name, regs in hits:
+            regs = int(regs)
+            low_threads = 128
+            need = low_threads * want["kRegsLow"] + (threads - low_threads) * want["kRegsHigh"]
+            if regs != want["kLaunchRegs"] or need > threads * regs:
+                raise RuntimeError(f"{name}: ptxas gives {regs} registers per thread at launch; the source assumes "
+                                   f"{want['kLaunchRegs']} and a split needing {need} of {threads * regs}")
 
 
 def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) -> str:
