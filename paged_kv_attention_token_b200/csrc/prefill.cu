@@ -71,8 +71,11 @@ constexpr float kPrefillRescaleThreshold = 8.f;
 // kPolyPairMask, a polynomial on the FMA and integer pipes.  The MUFU unit
 // does 16 results per SM clock, so 128 x 128 exponentials per head and
 // 128-key step take as long as that step's MMAs; moving part of them to the
-// FMA pipe shortens each softmax chain.
+// FMA pipe shortens each softmax chain.  Measured on B200: the two-head
+// kernel is fastest with the MUFU unit alone; the pair kernel gains ~2 %
+// with a quarter of the pairs on the polynomial (half of them: slower).
 constexpr uint32_t kPolyPairMask = 0x0;
+constexpr uint32_t kPairPolyPairMask = 0x1;
 // P is packed to bf16 pairs either with cvt.rn.bf16x2.f32 or with integer
 // adds and a byte permute (rounding half up; it differs from round-to-even
 // only on exact ties).
@@ -224,13 +227,14 @@ __device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], bool masked,
 
 // P for 32 S columns: 2^(s*scale - m) as 16 packed bf16 pairs; keys past
 // `pos` (when `masked`) get P = 0 by selection.
+template <uint32_t PolyMask = kPolyPairMask>
 __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], uint32_t (&pk)[16], uint64_t scale2,
                                           uint64_t nm2, bool masked, int key0, int pos) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint64_t x = f2_fma(f2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), scale2, nm2);
         float e0, e1;
-        if ((kPolyPairMask >> (c & 3)) & 1u) {
+        if ((PolyMask >> (c & 3)) & 1u) {
             f2_split(exp2_poly(x), e0, e1);
             if (masked) {
                 if (key0 + 2 * c > pos) e0 = 0.f;
@@ -978,9 +982,9 @@ __device__ __forceinline__ void pair_softmax_tile(const PrefillParams &p, const 
         }
         const uint64_t nm2 = f2(-m, -m);
         uint32_t pk0[16], pk1[16];
-        chunk_exp(s0, pk0, scale2, nm2, masked, kbase, pos);
+        chunk_exp<kPairPolyPairMask>(s0, pk0, scale2, nm2, masked, kbase, pos);
         tmem_st16(trow + s_col, pk0);
-        chunk_exp(s1, pk1, scale2, nm2, masked, kbase + 32, pos);
+        chunk_exp<kPairPolyPairMask>(s1, pk1, scale2, nm2, masked, kbase + 32, pos);
         tmem_st16(trow + s_col + 16, pk1);
         // O_half is rescaled after the previous step's PV product for this
         // half completed and before this step's P is handed over
