@@ -171,8 +171,10 @@ typedef struct {
     int64_t prefill_causal_pairs; /* (query, visible key) pairs per query head */
     uint64_t table_bytes;         /* the plan's device tables (uploaded once per build) */
     uint64_t workspace_bytes;     /* = pa_plan_workspace_bytes */
-    int32_t num_staged_kv_tiles;  /* 128-key K/V tiles of prefill segments gathered
-                                     into the workspace (per kv head) */
+    int32_t num_staged_kv_tiles;  /* 128-key K/V tiles gathered into the workspace
+                                     (per kv head): those of the prefill
+                                     segments, and of shared prefixes unless the
+                                     pair kernel reads those from the cache */
     int32_t num_prefill_ctas;     /* persistent CTAs of the prefill kernel */
     int32_t num_prefix_groups;    /* shared-prefix runs found (h_block_tables given) */
     int32_t attention_launches;   /* kernels one pa_attention_varlen call launches

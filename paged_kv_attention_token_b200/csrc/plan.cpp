@@ -428,6 +428,9 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
         cascade_choice = choose_cascade(p->num_sms, G, Hkv, groups, other_total, other_max,
                                         decode_cost_blocks * pa::kBlockSize * d.head_dim * 2 * 2, pair);
     }
+    // key tiles of the prefill segments: the staging list's head; a shared
+    // prefix's tiles follow (the pair kernel reads those from the paged cache)
+    const size_t seg_stages = stages.size();
     for (size_t k = 0; k < groups.size(); ++k) {
         const PrefixGroup &gr = groups[k];
         const int keys = gr.blocks * pa::kBlockSize;
@@ -576,7 +579,9 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     for (const pa::DecodeRow &r : rows) p->decode_keys += r.n_keys - (int64_t)r.first_block * pa::kBlockSize;
     p->num_tiles = (int32_t)tiles.size();
     p->num_prefill_ctas = p->prefill_pair ? 2 * grid : grid;
-    p->num_stages = (int32_t)stages.size();
+    // tiles the staging kernel gathers into the workspace (the list's head
+    // with the pair kernel, all of it otherwise)
+    p->num_stages = (int32_t)(p->prefill_pair ? seg_stages : stages.size());
 
     pa::TableLayout &t = p->tl;
     size_t off = 0;
@@ -598,7 +603,7 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     off = align_up(off + sizeof(float) * 2 * (size_t)piece_base * p->group, pa::kWorkspaceAlign);
     off = align_up(off, pa::kStagedAlign);
     w.staged = off;
-    off += stages.size() * 2 * (size_t)pa::kPrefillTileN * d.head_dim * 2;
+    off += (size_t)p->num_stages * 2 * (size_t)pa::kPrefillTileN * d.head_dim * 2;
     w.total = align_up(off, pa::kWorkspaceAlign);
 
     {

@@ -149,7 +149,7 @@ struct pa_plan {
     int32_t overlap_sms = 0;             // > 0: prefill runs on this many SMs beside the decode kernel
     bool cascade = false;                // shared-prefix tiles: the prefill kernel runs first
     int32_t num_prefix_groups = 0;
-    int32_t num_stages = 0;              // staged K/V key tiles
+    int32_t num_stages = 0;              // K/V key tiles staged into the workspace
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::TableLayout tl;
     pa::WorkspaceLayout ws;

@@ -405,6 +405,9 @@ __device__ __forceinline__ void softmax_tile(const PrefillParams &p, int nkv, in
 struct PrefillMaps {
     CUtensorMap q;
     CUtensorMap out;  // the same shape over the output (pair kernel's stores)
+    // pair kernel: the K and V caches as [blocks * 16][Hkv][D], box {64, 1, 16}
+    // (one 16-token block of one kv head, one 64-dim slab), 128-byte swizzle
+    CUtensorMap k, v;
 };
 
 // Gathers staged tile blockIdx.x (K for blockIdx.y = 0, V for 1) from the
@@ -1251,9 +1254,16 @@ __global__ void __launch_bounds__(384, 1)
             if (!mbar_wait(drain, 0, p.wait_limit)) err = true;
         } else if (warp == 1 && lane == 0) {
             // ------------------------------------------------ loads (both CTAs)
-            // In the order the MMAs consume them, per tile: Q, K0 K1 K2, V0 K3
-            // V1 K4 ...  A stage is reloaded once the MMAs that read it (in both
-            // CTAs) completed.
+            // In the order the MMAs consume them, per tile: Q, K0 K1, V0 K2,
+            // V1 K3 ...  A stage is reloaded once the MMAs that read it (in both
+            // CTAs) completed.  A prefill segment's K/V come from its staged
+            // tiles (bulk copies of this CTA's halves); a shared prefix's
+            // straight from the paged cache, one TMA box per 16-token block
+            // and 64-dim slab at the block's id from the block table, blocks
+            // past the keys not loaded (the forwarder zeroes what the V tile
+            // needs zeroed).  Staging pays where many query tiles read the
+            // same keys (a segment's); a prefix's tiles read each key tile
+            // once per head pair.
             int vs = 0, ks = 0;
             uint32_t vuse = 0, kuse = 0;
             for (int ti = t_begin; ti < t_end; ++ti) {
@@ -1267,62 +1277,125 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int s = 0; s < D / 64; ++s)
                     tma_load_3d(sQ + s * 16384, &maps.q, q_land, 64 * s, tile.head + (int)rank, tok0);
-                const uint8_t *kv = p.staged + (size_t)(tile.kv_base + tile.kv_tile0) * 2 * C::kTileBytes;
-                auto load_k = [&](const uint8_t *kt) {
+                // the keys' segment (or shared prefix), kv head and length
+                const bool gather = tile.row_base >= 0;
+                const StageTile src = p.stages[tile.kv_base];
+                const int32_t *bt = p.block_tables + (size_t)src.seq * p.max_blocks_per_seq;
+                const int nblk = (src.n_keys + kBlockSize - 1) / kBlockSize;
+                const uint8_t *kv = p.staged + (size_t)tile.kv_base * 2 * C::kTileBytes;  // segments only
+                auto load_k = [&](int t) {  // key tile t: this CTA's keys 64 rank .. + 63
                     if (kuse >= (uint32_t)C::kKStages && !err &&
                         !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1u, p.wait_limit))
                         err = true;
-                    mbar_arrive_expect_tx(&k_land[ks], C::kKBytes);
-                    // keys 64 rank .. + 63 of both 64-dim slabs
+                    if (!gather) {
+                        const uint8_t *kt = kv + (size_t)t * 2 * C::kTileBytes;
+                        mbar_arrive_expect_tx(&k_land[ks], C::kKBytes);
 #pragma unroll
-                    for (int s = 0; s < D / 64; ++s)
-                        bulk_load(sK + ks * C::kKBytes + s * 8192, kt + s * 16384 + rank * 8192, 8192, &k_land[ks]);
+                        for (int s = 0; s < D / 64; ++s)
+                            bulk_load(sK + ks * C::kKBytes + s * 8192, kt + s * 16384 + rank * 8192, 8192,
+                                      &k_land[ks]);
+                        ++kuse;
+                        if (++ks == C::kKStages) ks = 0;
+                        return;
+                    }
+                    const int b0 = 8 * t + 4 * (int)rank;
+                    int id[4];
+                    uint32_t bytes = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        id[i] = b0 + i < nblk ? __ldg(bt + b0 + i) : 0;
+                        bytes += b0 + i < nblk ? 2 * 2048 : 0;
+                    }
+                    mbar_arrive_expect_tx(&k_land[ks], bytes);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (b0 + i < nblk)
+#pragma unroll
+                            for (int s = 0; s < D / 64; ++s)
+                                tma_load_3d(sK + ks * C::kKBytes + s * 8192 + i * 2048, &maps.k, &k_land[ks], 64 * s,
+                                            src.kv_head, id[i] * kBlockSize);
                     ++kuse;
                     if (++ks == C::kKStages) ks = 0;
                 };
-                auto load_v = [&](const uint8_t *vt) {
+                auto load_v = [&](int t) {  // key tile t: dims 64 rank .. + 63 of its 128 keys
                     if (vuse >= (uint32_t)C::kVStages && !err &&
                         !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1u, p.wait_limit))
                         err = true;
-                    mbar_arrive_expect_tx(&v_land[vs], C::kVBytes);
-                    bulk_load(sV + vs * C::kVBytes, vt + rank * 16384, C::kVBytes, &v_land[vs]);  // dims 64 rank ..
+                    if (!gather) {
+                        const uint8_t *vt = kv + ((size_t)t * 2 + 1) * C::kTileBytes;
+                        mbar_arrive_expect_tx(&v_land[vs], C::kVBytes);
+                        bulk_load(sV + vs * C::kVBytes, vt + rank * 16384, C::kVBytes, &v_land[vs]);
+                        ++vuse;
+                        if (++vs == C::kVStages) vs = 0;
+                        return;
+                    }
+                    const int b0 = 8 * t;
+                    int id[8];
+                    uint32_t bytes = 0;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        id[i] = b0 + i < nblk ? __ldg(bt + b0 + i) : 0;
+                        bytes += b0 + i < nblk ? 2048 : 0;
+                    }
+                    mbar_arrive_expect_tx(&v_land[vs], bytes);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (b0 + i < nblk)
+                            tma_load_3d(sV + vs * C::kVBytes + i * 2048, &maps.v, &v_land[vs], 64 * (int)rank,
+                                        src.kv_head, id[i] * kBlockSize);
                     ++vuse;
                     if (++vs == C::kVStages) vs = 0;
                 };
-                for (int j = 0; j < C::kSBufs && j < n; ++j) load_k(kv + (size_t)j * 2 * C::kTileBytes);
+                for (int j = 0; j < C::kSBufs && j < n; ++j) load_k(tile.kv_tile0 + j);
                 for (int j = 0; j < n; ++j) {
-                    load_v(kv + ((size_t)j * 2 + 1) * C::kTileBytes);
-                    if (j + C::kSBufs < n) load_k(kv + (size_t)(j + C::kSBufs) * 2 * C::kTileBytes);
+                    load_v(tile.kv_tile0 + j);
+                    if (j + C::kSBufs < n) load_k(tile.kv_tile0 + j + C::kSBufs);
                 }
             }
-        } else if (warp == 2 && lane == 0) {
-            // ------------------------------------------------ forwarder (both CTAs)
+        } else if (warp == 2) {
+            // ------------------------------------------------ forwarder (both CTAs, one warp)
             // Walks the loads in the loader's order; once this CTA's copy has
-            // landed it arrives on rank 0's ready barrier.  Having waited for
-            // every landing, it also guarantees that no copy into this CTA is
-            // in flight when the CTA ends.
+            // landed it arrives on rank 0's ready barrier.  A V tile that
+            // reaches past the keys first gets its rows from the last key on
+            // zeroed (the blocks past the keys were not loaded, and the last
+            // block's slots past the keys may hold anything, NaN included,
+            // which P = 0 would not cancel).  Having waited for every landing,
+            // the warp also guarantees that no copy into this CTA is in
+            // flight when the CTA ends.
             int vs = 0, ks = 0;
             uint32_t vuse = 0, kuse = 0;
             auto fwd = [&](uint64_t *land, uint64_t *ready, uint32_t parity) {
                 if (!mbar_wait(land, parity, p.wait_limit)) err = true;
-                mbar_arrive_remote(at_rank0(ready));
+                if (lane == 0) mbar_arrive_remote(at_rank0(ready));
             };
             auto fwd_k = [&]() {
                 fwd(&k_land[ks], &k_ready[ks], (kuse / C::kKStages) & 1u);
                 ++kuse;
                 if (++ks == C::kKStages) ks = 0;
             };
-            auto fwd_v = [&]() {
-                fwd(&v_land[vs], &v_ready[vs], (vuse / C::kVStages) & 1u);
+            auto fwd_v = [&](int keys) {  // keys of the tile that exist (<= 128)
+                if (!mbar_wait(&v_land[vs], (vuse / C::kVStages) & 1u, p.wait_limit)) err = true;
+                if (keys < 128) {
+                    const uint32_t stage = sV + vs * C::kVBytes;
+                    for (int c = keys * 8 + lane; c < 128 * 8; c += 32)  // 16-byte chunks of 128-byte rows
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(stage + 16 * c), "r"(0u)
+                                     : "memory");
+                    fence_proxy_async_smem();  // the zeros, before the tensor cores read the tile
+                    __syncwarp();
+                }
+                if (lane == 0) mbar_arrive_remote(at_rank0(&v_ready[vs]));
                 ++vuse;
                 if (++vs == C::kVStages) vs = 0;
             };
             for (int ti = t_begin; ti < t_end; ++ti) {
-                const int n = p.tiles[ti].n_kv_tiles;
+                const PrefillTile tile = p.tiles[ti];
+                const int n = tile.n_kv_tiles;
+                // (staged tiles have their rows past the keys zeroed already)
+                const int n_keys = tile.row_base >= 0 ? p.stages[tile.kv_base].n_keys : 1 << 30;
                 fwd(q_land, q_ready, (uint32_t)(ti - t_begin) & 1u);
                 for (int j = 0; j < C::kSBufs && j < n; ++j) fwd_k();
                 for (int j = 0; j < n; ++j) {
-                    fwd_v();
+                    fwd_v(min(128, n_keys - 128 * (tile.kv_tile0 + j)));
                     if (j + C::kSBufs < n) fwd_k();
                 }
             }
@@ -1396,6 +1469,12 @@ cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
     const cuuint32_t box[3] = {64, 1, 128};
     if (!encode_bf16(enc, &maps.q, p.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
     if (!encode_bf16(enc, &maps.out, p.out, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    const cuuint64_t kv_dims[3] = {D, (cuuint64_t)p.num_kv_heads, (cuuint64_t)p.num_blocks * kBlockSize};
+    const cuuint64_t kv_strides[2] = {D * 2ull, (cuuint64_t)p.num_kv_heads * D * 2};
+    const cuuint32_t kv_box[3] = {64, 1, kBlockSize};
+    if (!encode_bf16(enc, &maps.k, p.k_cache, 3, kv_dims, kv_strides, kv_box) ||
+        !encode_bf16(enc, &maps.v, p.v_cache, 3, kv_dims, kv_strides, kv_box))
+        return cudaErrorInvalidValue;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaGetDevice(&dev);

@@ -74,12 +74,13 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_lib):
 def test_noalloc_rejects_plans_beyond_its_array(cuda_lib):
     lib = pa.load_library()
     cap = int(lib.pa_noalloc_scratch_bytes())
-    # one 8192-token prompt with 8 kv heads of 128 dims stages 64 key tiles of
-    # K and V per kv head in the scratch: 32 MiB
+    # one 8192-token prompt with 8 kv heads of 128 dims and an odd group (3
+    # query heads per kv head: the two-head kernel, which reads staged K/V)
+    # stages 64 key tiles of K and V per kv head in the scratch: 32 MiB
     S, n = 1, 8192
     cu = np.array([0, n], dtype=np.int32)
     sl = np.array([n], dtype=np.int32)
-    d = pa.Dims(n, S, 64, 8, 128, 1024, n // 16, 16)
+    d = pa.Dims(n, S, 24, 8, 128, 1024, n // 16, 16)
     plan = pa.Plan(cu, sl, d)
     assert plan.workspace_bytes > cap
     fake = ctypes.c_void_p(0x10000)         # never used: the call is rejected first
