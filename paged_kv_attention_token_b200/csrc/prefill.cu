@@ -1039,19 +1039,42 @@ __device__ __forceinline__ void pair_softmax_tile(const PrefillParams &p, const 
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive_remote(o_free0);
     if (tile.row_base >= 0) {
+        // Partials of decode rows, one row per thread, each row's 64 values at
+        // its own slot: they go out through a 4 KB region of the output
+        // staging per warp, 32 dims at a time, so that each store instruction
+        // writes four rows' whole 128-byte pieces instead of 32 scattered
+        // 16-byte ones.
+        const int G = p.group;
+        float *po = nullptr;
         if (t < q_rows) {
-            const int G = p.group;
             const int r = tile.row_base + t * p.num_kv_heads;
             const int slot = p.combine[p.rows[r].combine].piece_base + tile.piece;
-            float *po = p.partial_o + ((size_t)slot * G + hl) * D + kHalfO * half;
-#pragma unroll
-            for (int i = 0; i < kHalfO / 32; ++i)
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    reinterpret_cast<float4 *>(po + 32 * i)[c] =
-                        make_float4(__uint_as_float(o[i][4 * c]), __uint_as_float(o[i][4 * c + 1]),
-                                    __uint_as_float(o[i][4 * c + 2]), __uint_as_float(o[i][4 * c + 3]));
+            po = p.partial_o + ((size_t)slot * G + hl) * D + kHalfO * half;
             if (half == 0) p.partial_ml[(size_t)slot * G + hl] = make_float2(mm, lsum);
+        }
+        const bool issuer = (threadIdx.x & 127) == 0;
+        if (issuer) bulk_wait_read();  // a previous tile's output store has read the staging
+        named_sync(5 + half, 128);
+        const int lane = threadIdx.x & 31;
+        const uint32_t region = out_stage + ((threadIdx.x >> 5) - 4) * 4096;
+#pragma unroll
+        for (int i = 0; i < kHalfO / 32; ++i) {
+            // row `lane` of the warp: 32 floats, 16-byte chunk c at c ^ (lane % 8)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(region + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                             "r"(o[i][4 * c]), "r"(o[i][4 * c + 1]), "r"(o[i][4 * c + 2]), "r"(o[i][4 * c + 3])
+                             : "memory");
+            __syncwarp();
+#pragma unroll
+            for (int s4 = 0; s4 < 8; ++s4) {
+                const int row = 4 * s4 + (lane >> 3), c = lane & 7;
+                float *dst = reinterpret_cast<float *>(
+                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(po), row));
+                const uint4 v = ld_shared16(region + row * 128 + ((c ^ (row & 7)) << 4));
+                if (dst != nullptr) st16(dst + 32 * i + 4 * c, v);
+            }
+            __syncwarp();
         }
         return;
     }
