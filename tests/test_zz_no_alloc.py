@@ -30,13 +30,14 @@ def _dims(lay):
                    lay.head_dim, lay.num_blocks, lay.max_blocks_per_seq, 16)
 
 
-def _prepare(name, q_gain=1.0):
+def _prepare(name, q_gain=1.0, host_tables=False):
     lay = W.layout(name)
     b = W.make_batch(lay, device="cuda", q_gain=q_gain)
     kc, vc = b.k_cache.clone(), b.v_cache.clone()
     bt, cu, sl, slots = b.device_ints("cuda")
     pa.reshape_and_cache(b.k, b.v, slots, kc, vc)
-    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, _dims(lay))
+    plan = pa.Plan(lay.cu_seqlens_q, lay.seq_lens, _dims(lay),
+                   block_tables=lay.block_tables if host_tables else None)
     ws = pa.workspace_for(plan)
     ref = torch.full_like(b.q, float("nan"))
     pa.attention_varlen(b.q, kc, vc, bt, cu, sl, b.scale, ref, plan, ws)
@@ -52,7 +53,12 @@ def _call_noalloc(lib, b, kc, vc, bt, cu, sl, plan, out):
 
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_lib):
     lib = pa.load_library()
-    cases = [_prepare("decode_tinyllama_b64"), _prepare("tiny_mixed", q_gain=8.0)]
+    # the split-KV decode kernel; the two-head prefill kernel (head_dim 64);
+    # the pair kernel on staged prompts; the pair kernel on a shared prefix
+    # read from the paged cache, beside the decode kernel (partials, merges)
+    cases = [_prepare("decode_tinyllama_b64"), _prepare("tiny_mixed", q_gain=8.0),
+             _prepare("prefill_qwen25_1p5b_4x2048"), _prepare("prefix_llama3_70b_b128", host_tables=True)]
+    assert cases[2][6].info()["prefill_pair"] == 1 and cases[3][6].info()["num_prefix_groups"] == 1
     # two calls in a row per case, alternating cases, so each call starts from
     # the array contents the previous (different) call left behind
     for rnd in range(2):
