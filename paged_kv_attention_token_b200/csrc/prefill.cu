@@ -756,8 +756,9 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
 // The two-head kernel above keeps both heads of a tile in one SM's 512 TMEM
 // columns, so each head has a single S buffer and its loop S(j) -> softmax
 // -> PV(j) -> S(j + 1) is serial.  Here each SM holds one head: two S
-// buffers (256 columns) and O.  S(j + 2) is computed into the buffer P(j)
-// occupied, right after PV(j), so the softmax finds the next S ready.
+// buffers (256 columns) and two accumulators (below).  S(j + 2) is computed
+// into the buffer P(j) occupied, right after PV(j), so the softmax finds the
+// next S ready.
 //
 // A 2-SM MMA takes the 256 rows of A from both CTAs (rows 0-127 from rank 0,
 // 128-255 from rank 1: the two heads' Q in shared memory, or their P in
@@ -770,17 +771,24 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
 // beside the 1024 tensor cycles of the step's two products; a single SM
 // holding both heads moves 256 KB per two such steps.
 //
-// Rank 0 issues every MMA (one thread) and owns the barriers that gate them:
-// a K/V stage or Q is ready once a forwarding thread in each CTA has seen
-// that CTA's copy land and arrived on rank 0's barrier; P and the release of
-// O wait for the softmax warps of both CTAs (remote arrivals).  Every commit
+// Rank 0 issues every MMA (one warp, one elected lane) and owns the barriers
+// that gate them: a K/V stage or Q is ready once a forwarding warp in each
+// CTA has seen that CTA's copy land and arrived on rank 0's barrier; P and
+// the release of O wait for the softmax warps of both CTAs (remote
+// arrivals).  Every commit
 // arrives in both CTAs (tcgen05.commit cta_group::2 with cluster multicast),
 // so each CTA's loader, softmax warps and epilogue wait on barriers of their
 // own.  No TMA or bulk load uses cluster multicast.
 //
 // Eight softmax warps per CTA split every query row into two halves of 64
-// keys (warps 4-7 and 8-11 share TMEM lanes and exchange the half-row maxima
-// and sums through shared memory).
+// keys (warps 4-7 and 8-11 share TMEM lanes).  Each half is an online
+// softmax of its own, with its own running max and sum and its own
+// accumulator in TMEM (O_0 for keys 0-63 of every step, O_1 for 64-127), so
+// the two warps on an SM sub-partition never wait for each other within a
+// tile; the halves combine once per tile.
+//
+// A prefill segment's K/V come from staged tiles; a shared prefix's straight
+// from the paged cache (TMA boxes of one 16-token block), see the loader.
 // ---------------------------------------------------------------------------
 struct PairCfg {
     static constexpr int D = 128;
