@@ -582,17 +582,17 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
     if (!p.wait_first) grid_dependency_wait();
 }
 
-// Merges every combine row, one warp per row: used when the decode kernel
-// ran beside the kernel that writes a row's shared-prefix partials, so that
-// neither can merge.
+// Merges every combine row, one CTA per row (G x D / 8 items of one head
+// and 8 dims, 128 of them at G = 8, head_dim 128: one round of partial loads
+// per thread): used when
+// the decode kernel ran beside the kernel that writes a row's shared-prefix
+// partials, so that neither can merge.
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ DecodeParams p, int num_combine) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ci = blockIdx.x * 4 + warp;
-    if (ci >= num_combine) return;
+    const int ci = blockIdx.x;
     const CombineRow c = p.combine[ci];
     const DecodeRow row = p.rows[c.row];
-    merge_split_row<D>(p, c, row.token, (c.row % p.num_kv_heads) * p.group, lane, 32);
+    merge_split_row<D>(p, c, row.token, (c.row % p.num_kv_heads) * p.group, threadIdx.x, 128);
 }
 
 template <int D, int NT>
@@ -633,7 +633,7 @@ int decode_units_per_sm(int head_dim) {
 
 cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, cudaStream_t stream) {
     if (num_combine == 0) return cudaSuccess;
-    const int grid = (num_combine + 3) / 4;
+    const int grid = num_combine;
     if (head_dim == 64)
         merge_kernel<64><<<grid, 128, 0, stream>>>(p, num_combine);
     else
