@@ -227,11 +227,11 @@ __device__ __forceinline__ void attend_step(RowState<D, NT> &st, uint32_t stage,
 // Merge the partials of a split row and write it: O = sum_j 2^(m_j - M) O_j /
 // sum_j 2^(m_j - M) l_j with M = max_j m_j, in one pass with a running max.
 // Run by the warp that took the row's last ticket; the partials are read
-// through L2 (ld.cg), where the other warps' fenced writes are visible,
+// through L2 (ld.cg), where the other warps' released writes are visible,
 // kMergeBatch partials at a time so that the loads overlap instead of
 // forming a chain.
 template <int D>
-__device__ __noinline__ void merge_split_row(const DecodeParams &p, const CombineRow c, int token,
+__device__ __forceinline__ void merge_split_row(const DecodeParams &p, const CombineRow c, int token,
                                              int h0, int tid, int nthreads) {
     constexpr int kMergeBatch = 8;
     const int G = p.group;
@@ -283,6 +283,15 @@ __device__ __noinline__ void merge_split_row(const DecodeParams &p, const Combin
         o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
         st16(p.out + ((size_t)token * p.num_q_heads + h0 + head) * D + 8 * chunk, o);
     }
+}
+
+// Takes a ticket: returns the counter's old value and adds one, with release
+// semantics for the writes before it and acquire semantics for the reads
+// after it (GPU scope), in one round trip to L2.
+__device__ __forceinline__ uint32_t ticket_acq_rel(uint32_t *counter) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(counter) : "memory");
+    return old;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -563,15 +572,19 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
                     if (g8 == 0) p.partial_ml[(size_t)slot * G + head] = make_float2(st.m[nt][e], st.l[nt][e]);
                 }
             // publish the partial, take a ticket; the last warp of the row
-            // merges (unless a separate merge kernel follows)
-            __threadfence();
+            // merges (unless a separate merge kernel follows, which the
+            // kernel boundary orders after these writes).  The ticket is one
+            // acquire-release atomic of lane 0: the warp barrier before it
+            // orders every lane's partial writes before its release, and the
+            // one after it orders its acquire before every lane's reads of
+            // the other warps' partials.
             __syncwarp();
             if (p.defer_merge) return;
             int last = 0;
-            if (lane == 0) last = atomicAdd(&p.arrived[row.combine], 1u) == (uint32_t)c.tickets - 1;
+            if (lane == 0) last = ticket_acq_rel(&p.arrived[row.combine]) == (uint32_t)c.tickets - 1;
             last = __shfl_sync(kFullMask, last, 0);
             if (last) {
-                __threadfence();
+                __syncwarp();
                 merge_split_row<D>(p, c, row.token, h0, lane, 32);
                 // every ticket of this call is taken: leave the counter at zero
                 if (lane == 0) p.arrived[row.combine] = 0u;
