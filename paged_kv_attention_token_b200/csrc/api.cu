@@ -243,12 +243,33 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         pp.wait_limit = kWaitLimitCycles;
     }
     const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
-    if (side_by_side) {
-        // The prefill kernel (persistent, one CTA per SM, on overlap_sms SMs)
-        // stays on the caller's stream, runnable as soon as the staging
-        // kernel ends, so that its CTAs are placed first; the decode kernel,
-        // sized for the other SMs, waits on a side stream of the least
-        // priority for the fork event and fills those SMs.
+    if (side_by_side && !trace) {
+        // The prefill kernel (persistent, one CTA per SM or SM pair, on
+        // overlap_sms SMs) runs as soon as the staging kernel ends, so that
+        // its CTAs are placed first; each of them lets the dependent launch
+        // go as it starts.  The decode kernel, launched programmatically
+        // behind it on the same stream and sized for the other SMs, fills
+        // those SMs at once.  It reads nothing the staging or prefill
+        // kernels write (its inputs were complete before the staging kernel
+        // started), so it does not wait for them before its work, only at
+        // its end: what follows on the stream follows both.
+        if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        // shared-prefix partials are not ready while the decode kernel runs:
+        // it leaves every merge to the merge kernel behind both
+        p.defer_merge = plan->cascade ? 1 : 0;
+        p.wait_first = 0;
+        if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
+            return cuda_error();
+        if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
+            return cuda_error();
+        return PA_OK;
+    } else if (side_by_side) {
+        // Traced calls: the same two kernels side by side, with the decode
+        // kernel on a side stream of the least priority (forked after the
+        // staging kernel, joined before the merge), so that caller events
+        // can bracket each kernel on its own stream.
         cudaStream_t side = side_stream(plan->device);
         if (!side) return cuda_error();
         cudaEvent_t fork = static_cast<cudaEvent_t>(plan->fork_event);

@@ -459,6 +459,9 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *drain = bars + C::kBarDrain;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kTmemSlotOff);
 
+    // a decode kernel launched programmatically behind this one may place its
+    // CTAs on the other SMs now (it reads nothing this kernel writes)
+    grid_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (blockIdx.x >= p.num_ctas) return;
     const int t_begin = p.cta_start[blockIdx.x], t_end = p.cta_start[blockIdx.x + 1];
@@ -1156,6 +1159,9 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *o_done = bars + C::kBarO, *o_free = bars + C::kBarOFree, *drain = bars + C::kBarDrain;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kTmemSlotOff);
 
+    // a decode kernel launched programmatically behind this one may place its
+    // CTAs on the other SMs now (it reads nothing this kernel writes)
+    grid_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank();
     const int cl = blockIdx.x >> 1;
