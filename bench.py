@@ -363,8 +363,11 @@ def run_ours(args):
         flush.fill_(v)
         torch.sum(flush_read, dim=0, out=flush_sink)
     stream = torch.cuda.current_stream(dev)
-    # the scatter, then the kernels the attention call launches (plan info)
+    # the scatter, then the kernels the attention call launches (plan info);
+    # the fused call stages the prefill segments' keys in its scatter launch
     launches_per_step = (1 if lay.num_tokens else 0) + info["attention_launches"]  # scatter + attention
+    if not args.two_calls and lay.num_tokens and info["num_staged_kv_tiles"] > 0:
+        launches_per_step -= 1
 
     # two plans rebuilt in turn, as an engine keeps them across steps
     plan_pool = [pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt), pa.Plan(h_cu, h_sl, dims, device=local, block_tables=h_bt)]

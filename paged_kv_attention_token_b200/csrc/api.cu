@@ -170,7 +170,7 @@ int check_attention(const void *q, const void *k_cache, const void *v_cache, con
 int queue_attention(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                     const int32_t *cu_seqlens_q, const int32_t *seq_lens, float scale, void *out,
                     const pa_dims &d, const pa_plan *plan, void *workspace, void *stream_, const pa_trace *trace,
-                    const void *k_new, const void *v_new) {
+                    const void *k_new, const void *v_new, const ScatterArgs *scatter) {
     const WorkspaceLayout &w = plan->ws;
     const TableLayout &tl = plan->tl;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -242,6 +242,12 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         pp.scale_log2 = scale_log2;
         pp.wait_limit = kWaitLimitCycles;
     }
+    // A fused step starts with its cache write, and the staging of the
+    // prefill segments' keys runs in the same launch (their rows of this
+    // step's tokens taken from its K/V input): nothing of the staging is left
+    // in the branches below.
+    if (scatter && launch_scatter_stage(*scatter, pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+    if (scatter) pp.num_stages = 0;
     const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
     if (side_by_side && !trace) {
         // The prefill kernel (persistent, one CTA per SM or SM pair, on
@@ -334,7 +340,7 @@ extern "C" int pa_attention_varlen_ex(const void *q, const void *k_cache, const 
                                    workspace, workspace_bytes);
     if (st != PA_OK || dims->num_tokens == 0) return st;
     return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, *dims, plan,
-                           workspace, stream, trace, nullptr, nullptr);
+                           workspace, stream, trace, nullptr, nullptr, nullptr);
 }
 
 extern "C" int pa_reshape_and_attention(const void *k, const void *v, const int64_t *slot_mapping,
@@ -352,12 +358,18 @@ extern "C" int pa_reshape_and_attention(const void *k, const void *v, const int6
                                    workspace, workspace_bytes);
     if (st != PA_OK || dims->num_tokens == 0) return st;
     const pa_dims &d = *dims;
-    if (launch_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
-                                 (int64_t)d.num_blocks * d.block_size, current_sm_count(),
-                                 static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return cuda_error();
+    ScatterArgs sa{};
+    sa.k = k;
+    sa.v = v;
+    sa.slots = slot_mapping;
+    sa.k_cache = k_cache;
+    sa.v_cache = v_cache;
+    sa.num_tokens = d.num_tokens;
+    sa.token_elems = d.num_kv_heads * d.head_dim;
+    sa.num_slots = (int64_t)d.num_blocks * d.block_size;
+    sa.num_sms = current_sm_count();
     return queue_attention(q, k_cache, v_cache, block_tables, cu_seqlens_q, seq_lens, scale, out, d, plan,
-                           workspace, stream, nullptr, k, v);
+                           workspace, stream, nullptr, k, v, &sa);
 }
 
 namespace {

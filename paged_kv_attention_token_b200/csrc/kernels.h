@@ -79,6 +79,25 @@ struct PrefillParams {
 
 // Gathers the staged K/V tiles (must precede launch_prefill in stream order).
 cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stream);
+
+// A fused step's cache write: this step's K/V ([T][Hkv][D]) into their slots.
+struct ScatterArgs {
+    const void *k;
+    const void *v;
+    const int64_t *slots;
+    void *k_cache;
+    void *v_cache;
+    int64_t num_tokens;
+    int token_elems;   // Hkv * D
+    int64_t num_slots;  // blocks * 16
+    int num_sms;
+};
+// The cache write and the staging of p's tiles in one launch: the staged
+// rows of this step's own keys come from a.k / a.v, so neither part waits
+// for the other (every token's slot must be the cache position its segment's
+// block table gives it).  Without staged tiles, the plain scatter kernel.
+cudaError_t launch_scatter_stage(const ScatterArgs &a, const PrefillParams &p, int head_dim,
+                                 cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, int head_dim, cudaStream_t stream);
 
 // Self-test of the bounded-wait error path: one CTA holds tensor memory,

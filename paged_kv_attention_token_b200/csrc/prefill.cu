@@ -59,6 +59,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "scatter.cuh"
 
 namespace pa {
 
@@ -410,28 +411,69 @@ struct PrefillMaps {
     CUtensorMap k, v;
 };
 
-// Gathers staged tile blockIdx.x (K for blockIdx.y = 0, V for 1) from the
-// paged cache: 16-byte chunks, rows of one kv head's keys, swizzled as the
-// prefill kernel's shared-memory tiles.
+// Gathers staged tile `tile` (K for kv = 0, V for 1) from the paged cache:
+// 16-byte chunks, rows of one kv head's keys, swizzled as the prefill
+// kernel's shared-memory tiles; rows past the keys are zeroed.  With `fresh`
+// (a fused step's own K or V, [T][Hkv][D]), keys written by this step come
+// from it instead of their cache slots: key k of segment i is token
+// cu_seqlens_q[i] + k - (seq_lens[i] - q_len) when it is one of the last
+// q_len keys.
 template <int D>
-__global__ void __launch_bounds__(256) stage_kernel(const __grid_constant__ PrefillParams p) {
+__device__ __forceinline__ void stage_tile(const PrefillParams &p, int tile, int kv, const __nv_bfloat16 *fresh,
+                                           int tid, int nthreads) {
     constexpr int kRowChunks = D / 8;
-    const int kv = blockIdx.y;
-    const StageTile st = p.stages[blockIdx.x];
+    const StageTile st = p.stages[tile];
     const int n = st.n_keys;
     const int32_t *bt_row = p.block_tables + (size_t)st.seq * p.max_blocks_per_seq;
     const __nv_bfloat16 *cache = kv ? p.v_cache : p.k_cache;
-    uint8_t *tile = p.staged + ((size_t)blockIdx.x * 2 + kv) * (128 * D * 2);
-    for (int c = threadIdx.x; c < 128 * kRowChunks; c += 256) {
+    uint8_t *dst = p.staged + ((size_t)tile * 2 + kv) * (128 * D * 2);
+    int first_new = INT32_MAX, tok_base = 0;  // keys from first_new on are this step's tokens
+    if (fresh != nullptr) {
+        const int c0 = __ldg(p.cu_seqlens_q + st.seq), c1 = __ldg(p.cu_seqlens_q + st.seq + 1);
+        first_new = __ldg(p.seq_lens + st.seq) - (c1 - c0);
+        tok_base = c0 - first_new;
+    }
+    for (int c = tid; c < 128 * kRowChunks; c += nthreads) {
         const int row = c / kRowChunks, ch = c % kRowChunks;
         const int key = 128 * st.tile + row;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (key < n) {
-            const int blk = __ldg(bt_row + (key >> 4));
-            v = ld_stream16(cache + (((size_t)blk * kBlockSize + (key & 15)) * p.num_kv_heads + st.kv_head) * D + ch * 8);
+            if (key >= first_new) {
+                v = ld_stream16(fresh + ((size_t)(tok_base + key) * p.num_kv_heads + st.kv_head) * D + ch * 8);
+            } else {
+                const int blk = __ldg(bt_row + (key >> 4));
+                v = ld_stream16(cache + (((size_t)blk * kBlockSize + (key & 15)) * p.num_kv_heads + st.kv_head) * D +
+                                ch * 8);
+            }
         }
-        st16(tile + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4), v);
+        st16(dst + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4), v);
     }
+}
+
+// Gathers staged tile blockIdx.x (K for blockIdx.y = 0, V for 1).
+template <int D>
+__global__ void __launch_bounds__(256) stage_kernel(const __grid_constant__ PrefillParams p) {
+    stage_tile<D>(p, blockIdx.x, blockIdx.y, nullptr, threadIdx.x, 256);
+}
+
+// A fused step's cache write and staging in one launch: blocks below
+// scatter_blocks write this step's K/V into their slots, each block above
+// gathers one staged tile's K or V (its own keys from k / v).
+template <int D>
+__global__ void __launch_bounds__(256)
+    scatter_stage_kernel(const __grid_constant__ ScatterArgs a, const __grid_constant__ PrefillParams p,
+                         int scatter_blocks) {
+    // a decode kernel queued next may set up while this runs
+    grid_launch_dependents();
+    const int cpt = a.token_elems / 8;
+    if ((int)blockIdx.x < scatter_blocks) {
+        scatter_chunks(static_cast<const uint4 *>(a.k), static_cast<const uint4 *>(a.v), a.slots,
+                       static_cast<uint4 *>(a.k_cache), static_cast<uint4 *>(a.v_cache), a.num_tokens * cpt, cpt,
+                       a.num_slots, (int64_t)blockIdx.x * 256 + threadIdx.x, (int64_t)scatter_blocks * 256);
+        return;
+    }
+    const int i = blockIdx.x - scatter_blocks;
+    stage_tile<D>(p, i >> 1, i & 1, static_cast<const __nv_bfloat16 *>((i & 1) ? a.v : a.k), threadIdx.x, 256);
 }
 
 // One persistent CTA per SM works through its tiles [cta_start[c],
@@ -1548,6 +1590,22 @@ cudaError_t launch_stage(const PrefillParams &p, int head_dim, cudaStream_t stre
         stage_kernel<64><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
     else
         stage_kernel<128><<<dim3(p.num_stages, 2), 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_stage(const ScatterArgs &a, const PrefillParams &p, int head_dim,
+                                 cudaStream_t stream) {
+    if (p.num_stages == 0)
+        return launch_reshape_and_cache(a.k, a.v, a.slots, a.k_cache, a.v_cache, a.num_tokens, a.token_elems,
+                                        a.num_slots, a.num_sms, stream);
+    const int64_t chunks = a.num_tokens * (a.token_elems / 8);
+    // the scatter's share: as many blocks as the plain scatter kernel takes
+    const int scatter_blocks = (int)std::min<int64_t>((chunks + 255) / 256, (int64_t)a.num_sms * 8);
+    const dim3 grid(scatter_blocks + 2 * p.num_stages);
+    if (head_dim == 64)
+        scatter_stage_kernel<64><<<grid, 256, 0, stream>>>(a, p, scatter_blocks);
+    else
+        scatter_stage_kernel<128><<<grid, 256, 0, stream>>>(a, p, scatter_blocks);
     return cudaGetLastError();
 }
 

@@ -2,13 +2,11 @@
 // ("vLLM 学习笔记 01" §1.6: per token, the slot mapping names the block and
 // the row its K/V go to; slot = block_id * 16 + row).
 //
-// HBM-bound copy.  One thread moves one 16-byte chunk of one token's K (and
-// the same chunk of its V): a token's Hkv * D values are contiguous both in
-// k/v [T][Hkv][D] and in its cache row [NB][16][Hkv][D], so consecutive
-// threads read and write consecutive 16-byte chunks (full sectors on both
-// sides).  The grid is a whole number of waves over the SMs.
+// HBM-bound copy (scatter_chunks): one thread per 16-byte chunk of a token's
+// K and V.  The grid is a whole number of waves over the SMs.
 #include "common.cuh"
 #include "kernels.h"
+#include "scatter.cuh"
 
 namespace pa {
 
@@ -18,20 +16,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     int chunks_per_token, int64_t num_slots) {
     // an attention kernel queued next may set up while the copy runs
     grid_launch_dependents();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < num_chunks; c += stride) {
-        const int64_t t = c / chunks_per_token;
-        const int64_t part = c - t * chunks_per_token;
-        // the chunk's K/V do not depend on the slot: all three loads are in
-        // flight together, and only the stores wait for the slot
-        const int64_t s = __ldg(slots + t);
-        const uint4 kv = ld_stream16(k + c);
-        const uint4 vv = ld_stream16(v + c);
-        if (s < 0 || s >= num_slots) continue;  // negative: skip; past the pool: never written
-        const int64_t dst = s * chunks_per_token + part;
-        k_cache[dst] = kv;
-        v_cache[dst] = vv;
-    }
+    scatter_chunks(k, v, slots, k_cache, v_cache, num_chunks, chunks_per_token, num_slots,
+                   (int64_t)blockIdx.x * blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x);
 }
 
 cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t *slots,
