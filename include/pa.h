@@ -284,9 +284,11 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
  * equals pa_attention_varlen's bit for bit).  Cache write and attention
  * overlap: the decode kernel starts behind the scatter kernel by
  * programmatic launch and reads the keys of this step's own tokens from
- * d_k / d_v instead of their cache slots ("vLLM 学习笔记 01" §1.6: each new
+ * d_k / d_v instead of their cache slots, and the gather of the long
+ * segments' keys for the prefill kernel runs in the scatter's launch, taking
+ * those keys from d_k / d_v as well ("vLLM 学习笔记 01" §1.6: each new
  * token's K/V go to the slot its slot mapping names, and attention reads
- * them there; here the decode rows take the same values before they land).
+ * them there; here attention takes the same values before they land).
  * Precondition (besides those of both calls): every token t of segment i at
  * position p = seq_len - q_len + j has slot_mapping[t] ==
  * block_tables[i][p / 16] * 16 + p % 16, i.e. the slot mapping and the block
