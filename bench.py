@@ -27,7 +27,9 @@ time is the max over ranks.
 
 The JSON line adds: roofline (dominant kernel, timed in the same run with
 CUDA events around it on its stream, in a second pass of K identical steps,
-since event records cost GPU time of their own), the scatter kernel's own
+since event records cost GPU time of their own; for the decode kernel also
+a device copy of the same bytes timed the same way, what a plain copy
+reaches in one launch at that size), the scatter kernel's own
 roofline (back-to-back launches on distinct inputs and slots, after an L2
 flush), e2e (same metric through the public API with host buffers: after a
 flush and a synchronize, the host clock runs from before the step's plan
@@ -428,6 +430,30 @@ def run_ours(args):
     # (and, in a third pass, around the other stages of the call).
     peaks, peak_kind = load_peaks()
 
+    def copy_at_size(nbytes):
+        """A device copy moving the same bytes (half read, half written), timed
+        like the kernels (L2 flushed first, events on the stream): what one
+        launch of a plain copy reaches at this size, where fixed launch and
+        ramp costs weigh against the HBM rate of the peak (a large copy)."""
+        half = max(16, (nbytes // 2) // 16 * 16)
+        src = torch.ones(half, dtype=torch.uint8, device=dev)
+        dst = torch.empty(half, dtype=torch.uint8, device=dev)
+        times = []
+        for i in range(max(3, args.warmup) + max(5, args.steps)):
+            flush_l2(5)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dst.copy_(src)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= max(3, args.warmup):
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.mean(times)
+        gbs = 2 * half / (ms * 1e-3) / 1e9
+        del src, dst
+        return {"ms": ms, "gbs": gbs, "frac_of_peak": gbs / peaks["hbm_gbs"],
+                "how": "torch copy_ of the same bytes (half read, half written), L2 flushed, events, mean"}
+
     def traced_pass(stages):
         trs = [pa.Trace(stages=stages) for _ in range(args.steps)]
         for i in range(args.steps):
@@ -450,7 +476,9 @@ def run_ours(args):
                            "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
                            "frac": achieved / peaks["hbm_gbs"],
                            "traffic": profiled_traffic("decode_kernel", args.workload, src_hash),
-                           "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash}
+                           "algorithmic_bytes": dec_bytes, "ms": dec_ms, "source_hash": src_hash,
+                           "copy_at_size": copy_at_size(dec_bytes)}
+        roofline_decode["copy_at_size"]["decode_frac_of_it"] = achieved / roofline_decode["copy_at_size"]["gbs"]
     # when the plan runs the prefill kernel beside the decode kernel, it has
     # overlap_sms of the SMs: its peak is that share of the GPU's
     side_by_side = bool(info["num_decode_units"] and info["num_prefill_tiles"] and info["overlap_sms"] > 0)
@@ -520,7 +548,7 @@ def run_ours(args):
         per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in sc_ms) / nsets
         sc_bytes = 2 * (2 * T * Hkv * D * 2) + T * 8   # k, v read; cache rows written; slots read
         sc_gbs = sc_bytes / (per_launch_ms * 1e-3) / 1e9
-        sc_hash = kernel_source_hash(["scatter.cu", "common.cuh", "kernels.h", "plan.h"])
+        sc_hash = kernel_source_hash(["scatter.cu", "scatter.cuh", "common.cuh", "kernels.h", "plan.h"])
         scatter = {"bound": "hbm", "kernel": "reshape_and_cache_kernel", "achieved": sc_gbs,
                    "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
                    "frac": sc_gbs / peaks["hbm_gbs"],
