@@ -462,10 +462,11 @@ def run_ours(args):
         return [t.elapsed_ms() for t in trs]
 
     dec_ms = statistics.mean(s["decode"] for s in traced_pass(("decode",)))
-    other = traced_pass(("plan_wait", "combine", "prefill"))
+    other = traced_pass(("plan_wait", "combine", "staging", "prefill"))
     comb_ms = statistics.mean(s["combine"] for s in other)
     wait_ms = statistics.mean(s["plan_wait"] for s in other)
-    prefill_ms = statistics.mean(s["prefill"] for s in other)
+    prefill_ms = statistics.mean(s["prefill"] for s in other)  # the prefill kernel alone
+    staging_ms = statistics.mean(s["staging"] for s in other)
     split = decode_prefill_split(lay, info)
     roofline_decode = roofline_prefill = None
     dec_bytes = split["decode_bytes"]
@@ -497,6 +498,12 @@ def run_ours(args):
                             "traffic": profiled_traffic(prefill_kernel, args.workload, pre_hash),
                             "algorithmic_flops": split["prefill_flops"], "ms": prefill_ms,
                             "source_hash": pre_hash}
+        if not side_by_side and info["num_staged_kv_tiles"] > 0:
+            # the K/V staging kernel that precedes it (one extra read and write
+            # of the prefill segments' keys), timed in the same traced pass
+            roofline_prefill["staging_ms"] = staging_ms
+            roofline_prefill["frac_with_staging"] = split["prefill_flops"] / ((prefill_ms + staging_ms) * 1e-3) / 1e12 / \
+                (peaks["bf16_tflops"] * sm_share)
     # "roofline" is the dominant kernel's: the one with the longer device time
     # (side by side, both span about the step; the decode kernel, which
     # bounds the step through HBM, is reported)
@@ -675,6 +682,7 @@ def run_ours(args):
                        "step_api": ("pa_reshape_and_cache + pa_attention_varlen" if args.two_calls
                                     else "pa_reshape_and_attention"),
                        "stages_ms": {"plan_wait": wait_ms, "decode": dec_ms, "combine": comb_ms,
+                                     "staging": staging_ms if not side_by_side else None,
                                      "prefill": prefill_ms,
                                      "scatter": scatter["ms"] if scatter else None,
                                      "note": "separate traced passes; event records add GPU time"},

@@ -258,8 +258,10 @@ int pa_attention_varlen(const void *d_q, const void *d_k_cache, const void *d_v_
  *   [0] at the start of the call
  *   [1] before the split-KV decode kernel (which also merges split rows)
  *   [2] after the split-KV kernel      [3] = [2] (no separate combine kernel)
- *   [4] before the K/V staging and prefill kernels
+ *   [4] after the K/V staging kernel, before the prefill kernel
  *   [5] after the prefill kernel
+ * When the kernels run one after the other, the staging kernel runs between
+ * [3] and [4].
  * When the plan runs the two kernels side by side (pa_plan_info
  * num_prefill_ctas below the SM count while decode units exist), [1]-[3]
  * are recorded on the side stream that runs the decode kernel and [4], [5]

@@ -252,7 +252,9 @@ class Trace(ctypes.Structure):
     """Events recorded around the kernels of one attention call (pa_trace)."""
     _fields_ = [("events", ctypes.c_void_p * 6)]
 
-    MARKS = {"plan_wait": (0, 1), "decode": (1, 2), "combine": (2, 3), "prefill": (4, 5)}
+    # "staging" is the K/V staging kernel when the call runs its kernels one
+    # after the other (no decode kernel beside the prefill kernel)
+    MARKS = {"plan_wait": (0, 1), "decode": (1, 2), "combine": (2, 3), "staging": (3, 4), "prefill": (4, 5)}
 
     def __init__(self, stages=("plan_wait", "decode", "combine", "prefill")):
         """Record only the marks the named stages need (each record costs a

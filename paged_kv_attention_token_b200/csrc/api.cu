@@ -280,8 +280,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         if (!side) return cuda_error();
         cudaEvent_t fork = static_cast<cudaEvent_t>(plan->fork_event);
         cudaEvent_t join = static_cast<cudaEvent_t>(plan->join_event);
-        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
         if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
         if (cudaEventRecord(fork, stream) != cudaSuccess) return cuda_error();
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         if (cudaStreamWaitEvent(side, fork, 0) != cudaSuccess) return cuda_error();
@@ -301,8 +301,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         return PA_OK;
     } else if (plan->cascade) {
         // shared-prefix partials first; the decode kernel merges them
-        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
         if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         if (mark(trace, 5, stream) != cudaSuccess || mark(trace, 1, stream) != cudaSuccess) return cuda_error();
         if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
@@ -315,13 +315,10 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         // right behind the step's own scatter (fused step, no trace events)
         p.wait_first = k_new != nullptr && !trace ? 0 : 1;
         if (plan->num_units > 0 && launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
-        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess ||
-            mark(trace, 4, stream) != cudaSuccess)
-            return cuda_error();
-        if (plan->num_tiles > 0) {
-            if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
-            if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
-        }
+        if (mark(trace, 2, stream) != cudaSuccess || mark(trace, 3, stream) != cudaSuccess) return cuda_error();
+        if (plan->num_tiles > 0 && launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (mark(trace, 4, stream) != cudaSuccess) return cuda_error();
+        if (plan->num_tiles > 0 && launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
     }
     if (mark(trace, 5, stream) != cudaSuccess) return cuda_error();
     // the plan's next build waits for this
