@@ -242,6 +242,8 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         pp.scale_log2 = scale_log2;
         pp.wait_limit = kWaitLimitCycles;
     }
+    pp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    pp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
     // A fused step starts with its cache write, and the staging of the
     // prefill segments' keys runs in the same launch (their rows of this
     // step's tokens taken from its K/V input): nothing of the staging is left

@@ -57,6 +57,11 @@ struct PrefillParams {
     const int32_t *cta_start;  // CTA c owns tiles [cta_start[c], cta_start[c + 1])
     const StageTile *stages;   // the gather kernel's list
     uint8_t *staged;          // staged K/V tiles (workspace)
+    // a fused step's own K/V ([T][Hkv][D]), or null: with them, the pair
+    // kernel reads a segment's key tiles whose keys are all this step's
+    // tokens from here, and those tiles are not staged
+    const __nv_bfloat16 *k_new;
+    const __nv_bfloat16 *v_new;
     // shared-prefix tiles write partials of the decode rows they serve
     const DecodeRow *rows;
     const CombineRow *combine;

@@ -409,6 +409,10 @@ struct PrefillMaps {
     // pair kernel: the K and V caches as [blocks * 16][Hkv][D], box {64, 1, 16}
     // (one 16-token block of one kv head, one 64-dim slab), 128-byte swizzle
     CUtensorMap k, v;
+    // pair kernel, fused step: this step's K and V as [T][Hkv][D], box
+    // {64, 1, 64} (64 tokens of one kv head, one 64-dim slab), 128-byte
+    // swizzle: the layout of a staged tile's rows
+    CUtensorMap kn, vn;
 };
 
 // Gathers staged tile `tile` (K for kv = 0, V for 1) from the paged cache:
@@ -432,6 +436,8 @@ __device__ __forceinline__ void stage_tile(const PrefillParams &p, int tile, int
         const int c0 = __ldg(p.cu_seqlens_q + st.seq), c1 = __ldg(p.cu_seqlens_q + st.seq + 1);
         first_new = __ldg(p.seq_lens + st.seq) - (c1 - c0);
         tok_base = c0 - first_new;
+        // the pair kernel reads a tile of this step's keys only from the input
+        if (p.pair && 128 * st.tile >= first_new) return;
     }
     for (int c = tid; c < 128 * kRowChunks; c += nthreads) {
         const int row = c / kRowChunks, ch = c % kRowChunks;
@@ -774,7 +780,7 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     using C = PrefillCfg<D>;
     EncodeFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    PrefillMaps maps;
+    PrefillMaps maps{};
     const cuuint64_t dims[3] = {D, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.num_tokens};
     const cuuint64_t strides[2] = {D * 2ull, (cuuint64_t)p.num_q_heads * D * 2};
     const cuuint32_t box[3] = {64, 1, 128};
@@ -1362,10 +1368,30 @@ __global__ void __launch_bounds__(384, 1)
                 const int32_t *bt = p.block_tables + (size_t)src.seq * p.max_blocks_per_seq;
                 const int nblk = (src.n_keys + kBlockSize - 1) / kBlockSize;
                 const uint8_t *kv = p.staged + (size_t)tile.kv_base * 2 * C::kTileBytes;  // segments only
+                // a fused step: the segment's key tiles from first_new / 128 on
+                // hold only this step's tokens and come straight from its K/V
+                // input (key k is token key_tok + k), as 64-row boxes
+                int first_new = INT32_MAX, key_tok = 0;
+                if (!gather && p.k_new != nullptr) {
+                    const int c0 = p.cu_seqlens_q[tile.seq], c1 = p.cu_seqlens_q[tile.seq + 1];
+                    first_new = p.seq_lens[tile.seq] - (c1 - c0);
+                    key_tok = c0 - first_new;
+                }
+                const int kv_head = tile.head / p.group;
                 auto load_k = [&](int t) {  // key tile t: this CTA's keys 64 rank .. + 63
                     if (kuse >= (uint32_t)C::kKStages && !err &&
                         !mbar_wait(&k_empty[ks], (kuse / C::kKStages - 1) & 1u, p.wait_limit))
                         err = true;
+                    if (!gather && 128 * t >= first_new) {
+                        mbar_arrive_expect_tx(&k_land[ks], C::kKBytes);
+#pragma unroll
+                        for (int s = 0; s < D / 64; ++s)
+                            tma_load_3d(sK + ks * C::kKBytes + s * 8192, &maps.kn, &k_land[ks], 64 * s, kv_head,
+                                        key_tok + 128 * t + 64 * (int)rank);
+                        ++kuse;
+                        if (++ks == C::kKStages) ks = 0;
+                        return;
+                    }
                     if (!gather) {
                         const uint8_t *kt = kv + (size_t)t * 2 * C::kTileBytes;
                         mbar_arrive_expect_tx(&k_land[ks], C::kKBytes);
@@ -1400,6 +1426,16 @@ __global__ void __launch_bounds__(384, 1)
                     if (vuse >= (uint32_t)C::kVStages && !err &&
                         !mbar_wait(&v_empty[vs], (vuse / C::kVStages - 1) & 1u, p.wait_limit))
                         err = true;
+                    if (!gather && 128 * t >= first_new) {
+                        mbar_arrive_expect_tx(&v_land[vs], C::kVBytes);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(sV + vs * C::kVBytes + h * 8192, &maps.vn, &v_land[vs], 64 * (int)rank,
+                                        kv_head, key_tok + 128 * t + 64 * h);
+                        ++vuse;
+                        if (++vs == C::kVStages) vs = 0;
+                        return;
+                    }
                     if (!gather) {
                         const uint8_t *vt = kv + ((size_t)t * 2 + 1) * C::kTileBytes;
                         mbar_arrive_expect_tx(&v_land[vs], C::kVBytes);
@@ -1469,8 +1505,12 @@ __global__ void __launch_bounds__(384, 1)
             for (int ti = t_begin; ti < t_end; ++ti) {
                 const PrefillTile tile = p.tiles[ti];
                 const int n = tile.n_kv_tiles;
-                // (staged tiles have their rows past the keys zeroed already)
-                const int n_keys = tile.row_base >= 0 ? p.stages[tile.kv_base].n_keys : 1 << 30;
+                // (staged tiles have their rows past the keys zeroed already;
+                // a tile read from the step's input has the next tokens' rows
+                // there, or zeros past the input's end)
+                const int n_keys = tile.row_base >= 0 ? p.stages[tile.kv_base].n_keys
+                                   : p.k_new != nullptr ? p.seq_lens[tile.seq]
+                                                        : 1 << 30;
                 fwd(q_land, q_ready, (uint32_t)(ti - t_begin) & 1u);
                 for (int j = 0; j < C::kSBufs && j < n; ++j) fwd_k();
                 for (int j = 0; j < n; ++j) {
@@ -1542,7 +1582,7 @@ cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
     constexpr int D = C::D;
     EncodeFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    PrefillMaps maps;
+    PrefillMaps maps{};
     const cuuint64_t dims[3] = {D, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.num_tokens};
     const cuuint64_t strides[2] = {D * 2ull, (cuuint64_t)p.num_q_heads * D * 2};
     const cuuint32_t box[3] = {64, 1, 128};
@@ -1554,6 +1594,13 @@ cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
     if (!encode_bf16(enc, &maps.k, p.k_cache, 3, kv_dims, kv_strides, kv_box) ||
         !encode_bf16(enc, &maps.v, p.v_cache, 3, kv_dims, kv_strides, kv_box))
         return cudaErrorInvalidValue;
+    if (p.k_new != nullptr) {
+        const cuuint64_t new_dims[3] = {D, (cuuint64_t)p.num_kv_heads, (cuuint64_t)p.num_tokens};
+        const cuuint32_t new_box[3] = {64, 1, 64};
+        if (!encode_bf16(enc, &maps.kn, p.k_new, 3, new_dims, kv_strides, new_box) ||
+            !encode_bf16(enc, &maps.vn, p.v_new, 3, new_dims, kv_strides, new_box))
+            return cudaErrorInvalidValue;
+    }
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaGetDevice(&dev);

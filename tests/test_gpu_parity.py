@@ -334,6 +334,34 @@ def test_binding_rejects_wrong_dtypes(cuda_lib):
                             torch.empty_like(b.q), plan, ws)
 
 
+@pytest.mark.parametrize("name", ["mixed_qwen25_1p5b_t8192", "prefill_qwen25_1p5b_4x2048", "prefix_llama3_70b_b128"])
+def test_traced_call_matches_on_staged_and_side_by_side_plans(cuda_lib, name):
+    """A traced call runs the decode kernel on a side stream (side by side),
+    and records its marks around the staging and prefill kernels; its output
+    is the untraced call's bit for bit, and every interval is timed."""
+    lay = W.layout(name)
+    b = W.make_batch(lay, device="cuda")
+    kc, vc, ref, plan = run_step(b)
+    info = plan.info()
+    bt, cu, sl, _ = b.device_ints("cuda")
+    ws = pa.workspace_for(plan)
+    out = torch.full_like(b.q, float("nan"))
+    tr = pa.Trace(stages=("plan_wait", "decode", "combine", "staging", "prefill"))
+    pa.attention_varlen(b.q, kc, vc, bt, cu, sl, b.scale, out, plan, ws, trace=tr)
+    torch.cuda.synchronize()
+    assert pa.workspace_status(ws) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    t = tr.elapsed_ms()
+    assert t["prefill"] > 0 and all(t[k] >= 0 for k in ("plan_wait", "decode", "combine"))
+    if info["num_decode_units"] > 0:
+        assert t["decode"] > 0
+    # side by side, marks [3] and [4] are on different streams: the staging
+    # interval is defined only when the kernels run one after the other
+    side_by_side = info["overlap_sms"] > 0 and info["num_decode_units"] > 0
+    if not side_by_side and info["num_staged_kv_tiles"] > 0:
+        assert t["staging"] > 0
+
+
 def test_traced_call_matches_and_times_each_kernel(cuda_lib):
     lay = W.layout("decode_tinyllama_b64")
     b = W.make_batch(lay, device="cuda")
