@@ -248,8 +248,15 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
     // prefill segments' keys runs in the same launch (their rows of this
     // step's tokens taken from its K/V input): nothing of the staging is left
     // in the branches below.
-    if (scatter && launch_scatter_stage(*scatter, pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
-    if (scatter) pp.num_stages = 0;
+    // With the pair kernel and no tile of earlier keys to stage, the prefill
+    // kernel reads nothing the scatter writes: it starts behind it by
+    // programmatic launch and waits for it only at its end.
+    if (scatter) {
+        pp.wait_at_end = pp.pair && plan->num_stages_fused == 0 ? 1 : 0;
+        if (pp.wait_at_end) pp.num_stages = 0;  // the plain scatter kernel
+        if (launch_scatter_stage(*scatter, pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        pp.num_stages = 0;
+    }
     const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
     if (side_by_side && !trace) {
         // The prefill kernel (persistent, one CTA per SM or SM pair, on

@@ -80,6 +80,9 @@ struct PrefillParams {
     int max_blocks_per_seq;
     float scale_log2;
     long long wait_limit;  // SM cycles an mbarrier wait may take before the kernel gives up
+    // pair kernel launched programmatically behind a kernel it reads nothing
+    // of (a fused step's plain scatter): it waits for that kernel at its end
+    int wait_at_end;
 };
 
 // Gathers the staged K/V tiles (must precede launch_prefill in stream order).

@@ -582,6 +582,14 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     // tiles the staging kernel gathers into the workspace (the list's head
     // with the pair kernel, all of it otherwise)
     p->num_stages = (int32_t)(p->prefill_pair ? seg_stages : stages.size());
+    // a fused step with the pair kernel reads key tiles of the step's own
+    // tokens from its K/V input: only tiles with earlier keys are staged
+    p->num_stages_fused = 0;
+    for (size_t i = 0; i < seg_stages; ++i) {
+        const pa::StageTile &st = stages[i];
+        const int L = h_cu[st.seq + 1] - h_cu[st.seq];
+        if ((int64_t)pa::kPrefillTileN * st.tile < (int64_t)h_seq[st.seq] - L) ++p->num_stages_fused;
+    }
 
     pa::TableLayout &t = p->tl;
     size_t off = 0;

@@ -150,6 +150,8 @@ struct pa_plan {
     bool cascade = false;                // shared-prefix tiles: the prefill kernel runs first
     int32_t num_prefix_groups = 0;
     int32_t num_stages = 0;              // K/V key tiles staged into the workspace
+    int32_t num_stages_fused = 0;        // of them, those holding keys written before the step:
+                                         // the ones a fused step stages with the pair kernel
     int64_t prefill_pairs = 0;           // causal (query, key) pairs, per query head
     pa::TableLayout tl;
     pa::WorkspaceLayout ws;

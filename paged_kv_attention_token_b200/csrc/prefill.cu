@@ -1575,6 +1575,9 @@ __global__ void __launch_bounds__(384, 1)
     // MMAs, copies or arrivals may still touch it
     cluster_sync();
     if (warp == 0) tmem_dealloc_pair(tmem, C::kTmemCols);
+    // launched programmatically behind the step's scatter: what follows on
+    // the stream follows both
+    if (p.wait_at_end) grid_dependency_wait();
 }
 
 cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
@@ -1616,13 +1619,15 @@ cudaError_t launch_prefill_pair(const PrefillParams &p, cudaStream_t stream) {
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = p.wait_at_end ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_pair_kernel, p, maps);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
