@@ -288,7 +288,9 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
  * programmatic launch and reads the keys of this step's own tokens from
  * d_k / d_v instead of their cache slots, and the gather of the long
  * segments' keys for the prefill kernel runs in the scatter's launch, taking
- * those keys from d_k / d_v as well ("vLLM 学习笔记 01" §1.6: each new
+ * those keys from d_k / d_v as well (the two-SM prefill kernel reads key
+ * tiles of only this step's tokens from d_k / d_v directly, and starts
+ * behind the scatter when nothing else is gathered) ("vLLM 学习笔记 01" §1.6: each new
  * token's K/V go to the slot its slot mapping names, and attention reads
  * them there; here attention takes the same values before they land).
  * Precondition (besides those of both calls): every token t of segment i at
