@@ -12,7 +12,7 @@ import torch
 import paged_kv_attention_token_b200 as pa
 import workloads as W
 from tests.parity import assert_parity
-from tests.test_gpu_parity import CUSTOM, dims_for, gpu_rows, oracle_subset, run_step
+from tests.test_gpu_parity import CUSTOM, PREFILL, dims_for, gpu_rows, oracle_subset, run_step
 
 pytestmark = pytest.mark.gpu
 
@@ -80,6 +80,42 @@ def test_fused_spec_decode_against_oracle(cuda_lib, case, q_gain):
     check_against_two_calls(b)
 
 
+@pytest.mark.parametrize("case", range(len(PREFILL)))
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_fused_prefill_shapes_against_oracle(cuda_lib, case, q_gain):
+    # the prefill shapes through the fused call: with the two-SM kernel, key
+    # tiles of only the step's own tokens come straight from the K/V input
+    # (ragged last tiles included), chunks stage their earlier keys, and a
+    # plan with nothing left to stage starts the prefill kernel behind the
+    # scatter; every row against the oracle, and bit for bit the two calls
+    q_lens, seq_lens, Hq, Hkv, D = PREFILL[case]
+    nb = sum(-(-s // 16) for s in seq_lens) + 64
+    lay = W.custom_layout(q_lens, seq_lens, Hq, Hkv, D, nb, seed=200 + case)
+    b = W.make_batch(lay, device="cuda", q_gain=q_gain)
+    _, _, out, plan = run_fused(b)
+    tok, want = oracle_subset(b, range(lay.num_seqs))
+    assert_parity(gpu_rows(out, tok), want, f"fused prefill case {case} q_gain={q_gain} plan={plan.info()}")
+    check_against_two_calls(b)
+
+
+def test_fused_side_by_side_fresh_prompts(cuda_lib):
+    # decodes beside fresh prompts: the scatter, then the pair kernel by
+    # programmatic launch (nothing to stage), then the decode kernel behind
+    # it on the other SMs, each waiting for its predecessor only at its end
+    q = [1] * 300 + [1024, 512]
+    s = [2000] * 300 + [1024, 512]
+    nb = sum(-(-x // 16) for x in s) + 64
+    lay = W.custom_layout(q, s, 12, 2, 128, nb, seed=501)
+    b = W.make_batch(lay, device="cuda", q_gain=8.0)
+    _, _, out, plan = run_fused(b)
+    info = plan.info()
+    assert info["overlap_sms"] > 0 and info["prefill_pair"] == 1 and info["num_decode_units"] > 0
+    check_against_two_calls(b)
+    seqs = [0, 1, 150, 299, 300, 301]
+    tok, want = oracle_subset(b, seqs)
+    assert_parity(gpu_rows(out, tok), want, f"fused side by side, plan={info}")
+
+
 def test_fused_consecutive_calls_and_side_stream(cuda_lib):
     # the same step three times on one plan and workspace (merge tickets
     # reset, each scatter ordered after the previous call's kernels), on a
@@ -98,7 +134,7 @@ def test_fused_without_host_tables(cuda_lib):
 
 
 @pytest.mark.parametrize("name", ["tiny_mixed", "decode_tinyllama_b64", "prefix_llama3_70b_b128",
-                                  "mixed_qwen25_1p5b_t8192"])
+                                  "mixed_qwen25_1p5b_t8192", "prefill_qwen25_1p5b_4x2048"])
 def test_fused_step_captured_in_a_cuda_graph(cuda_lib, name):
     # the step (scatter + attention, one call) captured once and replayed:
     # decode only, shared prefix beside the suffix decode (merge kernel) and
