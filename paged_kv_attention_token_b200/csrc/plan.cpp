@@ -65,9 +65,13 @@ constexpr int64_t kRowCostBlocks = 8;
 // up to ~6.1 TB/s of HBM bandwidth (reached from ~92 SMs on).
 constexpr double kPrefillStepUs = 2.9;
 // The same step of a two-head tile on a cluster of two SMs (the pair kernel:
-// one head per SM, 2-SM MMAs), in microseconds of the cluster; measured on
-// B200 at ~1.22 on long chunks beside the decode kernel.
-constexpr double kPairStepUs = 1.25;
+// one head per SM, 2-SM MMAs), in microseconds of the cluster.  Measured on
+// B200 at ~1.22 on long chunks beside the decode kernel; 1.15 is what the
+// split is tuned with: on the 8192-token mixed step it gives the pair kernel
+// 36 SMs (499 us per fused step) where 1.05-1.10 / 1.20 / 1.25 / 1.35 give
+// 34 / 38 / 40 / 42 SMs (507 / 501 / 503 / 505 us), the decode kernel
+// finishing last in every case.
+constexpr double kPairStepUs = 1.15;
 constexpr double kDecodeBytesPerUsPerSm = 66e3;
 constexpr double kHbmBytesPerUs = 6.1e6;
 constexpr int kMinSideSms = 8;  // fewest SMs either kernel is given when they share the GPU
