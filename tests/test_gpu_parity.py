@@ -254,7 +254,8 @@ def test_full_size_decode_sampled(cuda_lib, name, q_gain):
 @pytest.mark.parametrize("q_gain", [1.0, 8.0])
 def test_full_size_mixed_sampled(cuda_lib, q_gain):
     """The 8192-token mixed step as bench.py runs it: the prefill kernel on
-    part of the SMs beside the decode kernel on the others (side stream).
+    part of the SMs beside the decode kernel on the others (launched behind
+    it on the same stream).
     Prefill rows are sampled at tile edges; 64 random decodes cover rows
     that the plan cuts between warps and rows it does not."""
     lay = W.layout("mixed_qwen25_1p5b_t8192")
