@@ -271,11 +271,13 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         if (launch_stage(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         if (launch_prefill(pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         // shared-prefix partials are not ready while the decode kernel runs:
-        // it leaves every merge to the merge kernel behind both
+        // it leaves every merge to the merge kernel behind both (launched
+        // programmatically: its CTAs become resident as the decode kernel
+        // ends, and wait for it before reading partials)
         p.defer_merge = plan->cascade ? 1 : 0;
         p.wait_first = 0;
         if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
-        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
+        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, true, stream) != cudaSuccess)
             return cuda_error();
         if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
             return cuda_error();
@@ -303,7 +305,7 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         if (mark(trace, 5, stream) != cudaSuccess) return cuda_error();  // prefill, not the join
         if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
             return cuda_error();
-        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, stream) != cudaSuccess)
+        if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, false, stream) != cudaSuccess)
             return cuda_error();
         if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)
             return cuda_error();

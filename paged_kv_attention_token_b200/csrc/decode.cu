@@ -599,12 +599,16 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
 // and 8 dims, 128 of them at G = 8, head_dim 128: one round of partial loads
 // per thread): used when
 // the decode kernel ran beside the kernel that writes a row's shared-prefix
-// partials, so that neither can merge.
+// partials, so that neither can merge.  Launched programmatically behind
+// the decode kernel, its CTAs read their plan entries while that kernel
+// ends and wait for it (and with it for the prefill kernel, which the
+// decode kernel waits for at its end) before reading any partial.
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ DecodeParams p, int num_combine) {
     const int ci = blockIdx.x;
     const CombineRow c = p.combine[ci];
     const DecodeRow row = p.rows[c.row];
+    grid_dependency_wait();
     merge_split_row<D>(p, c, row.token, (c.row % p.num_kv_heads) * p.group, threadIdx.x, 128);
 }
 
@@ -644,14 +648,21 @@ int decode_units_per_sm(int head_dim) {
                           : DecodeCfg<128, 1>::kWarps * DecodeCfg<128, 1>::kCtasPerSm;
 }
 
-cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, cudaStream_t stream) {
+cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, bool programmatic,
+                         cudaStream_t stream) {
     if (num_combine == 0) return cudaSuccess;
-    const int grid = num_combine;
-    if (head_dim == 64)
-        merge_kernel<64><<<grid, 128, 0, stream>>>(p, num_combine);
-    else
-        merge_kernel<128><<<grid, 128, 0, stream>>>(p, num_combine);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(num_combine);
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = programmatic ? 1 : 0;
+    const cudaError_t e = head_dim == 64 ? cudaLaunchKernelEx(&cfg, merge_kernel<64>, p, num_combine)
+                                         : cudaLaunchKernelEx(&cfg, merge_kernel<128>, p, num_combine);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream) {

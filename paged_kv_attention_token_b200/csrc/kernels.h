@@ -43,7 +43,11 @@ cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);
 // Merges all combine rows (after a decode launch with defer_merge).
-cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, cudaStream_t stream);
+// programmatic: launched with programmatic stream serialization right behind
+// that decode launch on the same stream (its CTAs wait for the decode kernel
+// in the kernel); otherwise a plain launch.
+cudaError_t launch_merge(const DecodeParams &p, int head_dim, int num_combine, bool programmatic,
+                         cudaStream_t stream);
 
 struct PrefillParams {
     const __nv_bfloat16 *q;
