@@ -92,7 +92,7 @@ extern "C" int pa_reshape_and_cache(const void *k, const void *v, const int64_t 
         return PA_ERR_ALIGN;
     const cudaError_t e = launch_reshape_and_cache(
         k, v, slot_mapping, k_cache, v_cache, d.num_tokens, d.num_kv_heads * d.head_dim,
-        (int64_t)d.num_blocks * d.block_size, current_sm_count(),
+        (int64_t)d.num_blocks * d.block_size, current_sm_count(), false,
         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : cuda_error();
 }
@@ -251,13 +251,23 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
     // With the pair kernel and no tile of earlier keys to stage, the prefill
     // kernel reads nothing the scatter writes: it starts behind it by
     // programmatic launch and waits for it only at its end.
-    if (scatter) {
+    const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
+    // When neither attention kernel reads what the scatter writes (the pair
+    // kernel with no tile of earlier keys to stage: every key it reads is an
+    // earlier one from the cache, or this step's from the K/V input, and so
+    // are the decode kernel's) and the two run side by side, the scatter is
+    // queued last: a scatter queued first holds registers on the SMs the
+    // prefill clusters need, and the decode launch waits until every
+    // prefill CTA has started.
+    const bool scatter_last =
+        scatter && side_by_side && !trace && pp.pair && plan->num_stages_fused == 0;
+    if (scatter && !scatter_last) {
         pp.wait_at_end = pp.pair && plan->num_stages_fused == 0 ? 1 : 0;
         if (pp.wait_at_end) pp.num_stages = 0;  // the plain scatter kernel
         if (launch_scatter_stage(*scatter, pp, d.head_dim, stream) != cudaSuccess) return cuda_error();
         pp.num_stages = 0;
     }
-    const bool side_by_side = plan->overlap_sms > 0 && plan->num_units > 0 && plan->num_tiles > 0;
+    if (scatter_last) pp.num_stages = 0;
     if (side_by_side && !trace) {
         // The prefill kernel (persistent, one CTA per SM or SM pair, on
         // overlap_sms SMs) runs as soon as the staging kernel ends, so that
@@ -276,7 +286,16 @@ int queue_attention(const void *q, const void *k_cache, const void *v_cache, con
         // ends, and wait for it before reading partials)
         p.defer_merge = plan->cascade ? 1 : 0;
         p.wait_first = 0;
+        // a scatter queued last starts beside the decode kernel (in the
+        // room its CTAs leave on their SMs) and waits for it at its end, so
+        // that what follows still follows all three
+        p.trigger_dependents = scatter_last ? 1 : 0;
         if (launch_decode(p, d.head_dim, stream) != cudaSuccess) return cuda_error();
+        if (scatter_last &&
+            launch_reshape_and_cache(scatter->k, scatter->v, scatter->slots, scatter->k_cache, scatter->v_cache,
+                                     scatter->num_tokens, scatter->token_elems, scatter->num_slots,
+                                     scatter->num_sms, true, stream) != cudaSuccess)
+            return cuda_error();
         if (p.defer_merge && launch_merge(p, d.head_dim, plan->num_combine, true, stream) != cudaSuccess)
             return cuda_error();
         if (track_use && cudaEventRecord(static_cast<cudaEvent_t>(plan->use_event), stream) != cudaSuccess)

@@ -463,6 +463,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, NT>::kThreads, DecodeCfg<D, NT>::
     // data depends on it, and the wait moves to the end (so that what
     // follows on the stream also follows the scatter).
     if (p.wait_first) grid_dependency_wait();
+    if (p.trigger_dependents) grid_launch_dependents();
 
     // Load cursor: this warp's next step to copy; S-1 steps run ahead.
     LoadCursor lc;

@@ -34,11 +34,17 @@ struct DecodeParams {
     const __nv_bfloat16 *k_new;
     const __nv_bfloat16 *v_new;
     int wait_first;             // 0 only right behind the step's own scatter (see decode_kernel)
+    // nonzero: lets the next launch on the stream (the step's own scatter,
+    // queued behind it) go as the kernel starts
+    int trigger_dependents;
 };
 
+// behind: launched programmatically behind the kernels of its own step (it
+// then starts as they let it and waits for them at its end); otherwise a
+// plain launch.
 cudaError_t launch_reshape_and_cache(const void *k, const void *v, const int64_t *slots,
                                      void *k_cache, void *v_cache, int64_t num_tokens,
-                                     int token_elems, int64_t num_slots, int num_sms,
+                                     int token_elems, int64_t num_slots, int num_sms, bool behind,
                                      cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, int head_dim, cudaStream_t stream);

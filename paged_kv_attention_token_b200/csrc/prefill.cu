@@ -1649,7 +1649,7 @@ cudaError_t launch_scatter_stage(const ScatterArgs &a, const PrefillParams &p, i
                                  cudaStream_t stream) {
     if (p.num_stages == 0)
         return launch_reshape_and_cache(a.k, a.v, a.slots, a.k_cache, a.v_cache, a.num_tokens, a.token_elems,
-                                        a.num_slots, a.num_sms, stream);
+                                        a.num_slots, a.num_sms, false, stream);
     const int64_t chunks = a.num_tokens * (a.token_elems / 8);
     // the scatter's share: as many blocks as the plain scatter kernel takes
     const int scatter_blocks = (int)std::min<int64_t>((chunks + 255) / 256, (int64_t)a.num_sms * 8);
