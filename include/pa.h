@@ -290,9 +290,14 @@ int pa_attention_varlen_ex(const void *d_q, const void *d_k_cache, const void *d
  * segments' keys for the prefill kernel runs in the scatter's launch, taking
  * those keys from d_k / d_v as well (the two-SM prefill kernel reads key
  * tiles of only this step's tokens from d_k / d_v directly, and starts
- * behind the scatter when nothing else is gathered) ("vLLM 学习笔记 01" §1.6: each new
+ * behind the scatter when nothing else is gathered; when it runs beside the
+ * decode kernel with nothing gathered, neither attention kernel reads the
+ * slots the scatter writes, and the scatter is queued after them instead,
+ * running beside the decode kernel) ("vLLM 学习笔记 01" §1.6: each new
  * token's K/V go to the slot its slot mapping names, and attention reads
  * them there; here attention takes the same values before they land).
+ * Everything queued on the stream after the call follows all of its
+ * kernels, whichever order they run in.
  * Precondition (besides those of both calls): every token t of segment i at
  * position p = seq_len - q_len + j has slot_mapping[t] ==
  * block_tables[i][p / 16] * 16 + p % 16, i.e. the slot mapping and the block
