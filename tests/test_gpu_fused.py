@@ -116,11 +116,13 @@ def test_fused_side_by_side_fresh_prompts(cuda_lib):
     assert_parity(gpu_rows(out, tok), want, f"fused side by side, plan={info}")
 
 
-def test_fused_consecutive_calls_and_side_stream(cuda_lib):
+@pytest.mark.parametrize("name", ["decode_tinyllama_b64", "prefix_llama3_70b_b128"])
+def test_fused_consecutive_calls_and_side_stream(cuda_lib, name):
     # the same step three times on one plan and workspace (merge tickets
-    # reset, each scatter ordered after the previous call's kernels), on a
-    # stream of its own
-    b = W.make_batch(W.layout("decode_tinyllama_b64"), device="cuda")
+    # reset, each call's kernels ordered after the previous call's: with the
+    # shared prefix, the scatter queued behind the side-by-side kernels and
+    # the programmatic merge launch), on a stream of its own
+    b = W.make_batch(W.layout(name), device="cuda")
     _, _, ref, _ = run_step(b)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
