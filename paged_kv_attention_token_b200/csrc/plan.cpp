@@ -57,6 +57,14 @@ constexpr int64_t kMinBlocksPerUnit = 4;
 // merge) and starting the next (its q) take about as long as streaming this
 // many blocks, so a run that crosses a row boundary gets fewer blocks.
 constexpr int64_t kRowCostBlocks = 8;
+// The same charge where runs are long (kLongRunBlocks blocks or more on
+// average): there a row's finish overlaps more of the run's streaming.
+// B200, fused steps: 256 requests of Llama-3-8B shape (~300 blocks per run)
+// 425.6-426.7 us with 4 against 429.6-431.2 with 8 (6: 429.0); 64 requests
+// of TinyLlama shape (~15 blocks per run) 23.6 us with 8 against 25.6 with
+// 4 (12-24: 23.6-24.0).  The threshold lies between the two.
+constexpr int64_t kRowCostBlocksLongRuns = 4;
+constexpr int64_t kLongRunBlocks = 64;
 
 // Cost model for running the prefill kernel beside the decode kernel on
 // disjoint SMs (B200 measurements): one 128-key step of a two-head tile
@@ -506,21 +514,22 @@ extern "C" int pa_plan_build(const int32_t *h_cu, const int32_t *h_seq, const in
     }
 
     // Cut the decode rows' blocks into equal runs of cost: each row's
-    // blocks, then kRowCostBlocks of virtual cost, laid end to end.
+    // blocks, then the per-row charge of virtual cost, laid end to end.
     const int64_t R = (int64_t)rows.size();
     std::vector<int64_t> prefix(R + 1, 0), nblocks(R, 0);
+    int64_t total = 0;  // real blocks
     for (int64_t r = 0; r < R; ++r) {
         nblocks[r] = cdiv(rows[r].n_keys, pa::kBlockSize) - rows[r].first_block;
-        prefix[r + 1] = prefix[r] + nblocks[r] + kRowCostBlocks;
+        total += nblocks[r];
     }
-    const int64_t total_cost = prefix[R];
-    int64_t total = 0;  // real blocks
-    for (int64_t r = 0; r < R; ++r) total += nblocks[r];
     int64_t P = 0;
     if (total > 0) {
         const int64_t max_units = (int64_t)decode_sms * pa::decode_units_per_sm(d.head_dim);
         P = std::max<int64_t>(1, std::min(max_units, cdiv(total, kMinBlocksPerUnit)));
     }
+    const int64_t row_cost = P > 0 && total / P >= kLongRunBlocks ? kRowCostBlocksLongRuns : kRowCostBlocks;
+    for (int64_t r = 0; r < R; ++r) prefix[r + 1] = prefix[r] + nblocks[r] + row_cost;
+    const int64_t total_cost = prefix[R];
     std::vector<pa::DecodeUnit> units(P + 1);
     std::vector<int64_t> ustart(P + 1);
     {
